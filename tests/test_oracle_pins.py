@@ -1,0 +1,151 @@
+"""The oracle passes every pin; copies with a planted mistake fail at least one.
+
+Planted mistakes live only here, in CPU code, on the oracle side."""
+import numpy as np
+import pytest
+
+from oracle import reference as ref
+import pins
+
+# ----------------------------------------------------------------------------
+# the real oracle passes
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("pin", pins.PATCHIFY_PINS, ids=lambda p: p.__name__)
+def test_patchify_pins(pin):
+    pin(ref.patchify)
+
+
+@pytest.mark.parametrize("pin", pins.ROPE_PINS, ids=lambda p: p.__name__)
+def test_rope_pins(pin):
+    pin(ref.rope_3d)
+
+
+@pytest.mark.parametrize("pin", pins.ATTENTION_PINS, ids=lambda p: p.__name__)
+def test_attention_pins(pin):
+    pin(lambda q, k, v, scale: ref.attention(q, k, v, scale))
+
+
+def test_divided_pins():
+    pins.pin_divided_time(ref.divided_time)
+    pins.pin_divided_space(ref.divided_space)
+    pins.pin_divided_degenerate(ref.divided_time, ref.divided_space)
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes are caught
+# ----------------------------------------------------------------------------
+
+
+def _fails(pin_list, fn):
+    caught = 0
+    for pin in pin_list:
+        try:
+            pin(fn)
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    return caught
+
+
+def patchify_feature_order_swapped(latent, pt, ph, pw):
+    """Mistake: brick features ordered (dt, dh, dw, c) instead of (c, dt, dh, dw)."""
+    N, C, T, H, W = latent.shape
+    Tg, Hg, Wg = T // pt, H // ph, W // pw
+    x = latent[:, :, :Tg * pt, :Hg * ph, :Wg * pw].reshape(N, C, Tg, pt, Hg, ph, Wg, pw)
+    return x.transpose(0, 2, 4, 6, 3, 5, 7, 1).reshape(N, Tg * Hg * Wg, -1)
+
+
+def patchify_token_order_swapped(latent, pt, ph, pw):
+    """Mistake: tokens flattened width-major instead of time-major."""
+    N, C, T, H, W = latent.shape
+    Tg, Hg, Wg = T // pt, H // ph, W // pw
+    x = latent[:, :, :Tg * pt, :Hg * ph, :Wg * pw].reshape(N, C, Tg, pt, Hg, ph, Wg, pw)
+    return x.transpose(0, 6, 4, 2, 1, 3, 5, 7).reshape(N, Tg * Hg * Wg, -1)
+
+
+@pytest.mark.parametrize("bad", [patchify_feature_order_swapped, patchify_token_order_swapped])
+def test_patchify_mistakes_caught(bad):
+    assert _fails(pins.PATCHIFY_PINS, bad) >= 1
+
+
+def _rope_variant(x, grid, split, theta=10000.0, freq_width=None, pairing="adjacent",
+                  sign=1.0, axis_order=(0, 1, 2)):
+    B, L, Hh, D = x.shape
+    ref.check_split(D, split)
+    Tg, Hg, Wg = grid
+    idx = np.arange(L)
+    pos = [idx // (Hg * Wg), (idx // Wg) % Hg, idx % Wg]
+    angs = []
+    for a, d in enumerate(split):
+        w = d if freq_width is None else freq_width
+        f = 1.0 / theta ** (np.arange(0, d, 2) / w)
+        angs.append(np.outer(pos[axis_order[a]], f))
+    ang = np.concatenate(angs, 1)
+    c, s = np.cos(ang)[None, :, None], np.sin(ang)[None, :, None]
+    out = np.empty_like(x)
+    if pairing == "adjacent":
+        i0, i1 = np.arange(0, D, 2), np.arange(1, D, 2)
+    else:  # rotate-half within each axis segment
+        i0, i1, off = [], [], 0
+        for d in split:
+            i0 += list(range(off, off + d // 2))
+            i1 += list(range(off + d // 2, off + d))
+            off += d
+        i0, i1 = np.array(i0), np.array(i1)
+    x0, x1 = x[..., i0], x[..., i1]
+    out[..., i0] = x0 * c - sign * x1 * s
+    out[..., i1] = sign * x0 * s + x1 * c
+    return out
+
+
+@pytest.mark.parametrize("kw", [
+    dict(freq_width=128),            # frequencies from the head width, not the axis width
+    dict(pairing="half"),            # rotate-half pairs instead of adjacent pairs
+    dict(sign=-1.0),                 # rotation in the wrong direction
+    dict(axis_order=(2, 1, 0)),      # width position on the time segment
+], ids=["head-width-freq", "rotate-half", "sign", "axis-order"])
+def test_rope_mistakes_caught(kw):
+    # the unmodified variant passes, so a failure below is the planted mistake
+    for pin in pins.ROPE_PINS:
+        pin(lambda x, g, s: _rope_variant(x, g, s))
+    bad = lambda x, g, s: _rope_variant(x, g, s, **kw)
+    assert _fails(pins.ROPE_PINS, bad) >= 1
+
+
+def _attention_variant(q, k, v, scale, no_scale=False, no_norm=False, drop_last_key=False):
+    B, L, H, D = q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    if no_scale:
+        scale = 1.0
+    o = np.empty_like(v)
+    lse = np.empty((B, H, L))
+    for b in range(B):
+        for h in range(H):
+            kk = k[b, :, h][:-1] if (drop_last_key and k.shape[1] > 1) else k[b, :, h]
+            vv = v[b, :, h][:-1] if (drop_last_key and k.shape[1] > 1) else v[b, :, h]
+            s = q[b, :, h] @ kk.T * scale
+            m = s.max(1, keepdims=True)
+            p = np.exp(s - m)
+            l = p.sum(1, keepdims=True)
+            o[b, :, h] = p @ vv if no_norm else (p @ vv) / l
+            lse[b, h] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+@pytest.mark.parametrize("kw", [dict(no_scale=True), dict(no_norm=True), dict(drop_last_key=True)],
+                         ids=["no-scale", "no-normalise", "ragged-tail-dropped"])
+def test_attention_mistakes_caught(kw):
+    for pin in pins.ATTENTION_PINS:
+        pin(_attention_variant)
+    bad = lambda q, k, v, s: _attention_variant(q, k, v, s, **kw)
+    assert _fails(pins.ATTENTION_PINS, bad) >= 1
+
+
+def test_divided_mistakes_caught():
+    # time pass that groups by frame (it is the space pass), and the reverse
+    with pytest.raises(AssertionError):
+        pins.pin_divided_time(lambda q, k, v, T, HW, s: ref.divided_space(q, k, v, T, HW, s))
+    with pytest.raises(AssertionError):
+        pins.pin_divided_space(lambda q, k, v, T, HW, s: ref.divided_time(q, k, v, T, HW, s))
