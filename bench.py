@@ -1,0 +1,429 @@
+"""Benchmark of the spacetime-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step runs every step of the path once on one batch of seeded synthetic
+input resident in HBM:
+
+    patchify (latent -> tokens) -> 3D RoPE on Q, K -> full 3D attention
+                                                   -> time pass + space pass
+
+The default workload is the 81-frame 832x480 clip as a CFG pair: latent
+[2, 16, 21, 60, 104] fp32, patch (1, 2, 2) -> 32,760 tokens, Q/K/V
+[2, 32760, 40, 128] bf16 ~ N(0, 1) (seed 0; the projection that would produce
+them needs trained weights and is not part of the path).  The metric is
+attention TFLOP/s over the step (4*L_q*L_k*D per head for every attention
+call; patchify and RoPE add time, no FLOPs) and ms per step (one layer).
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own clip pair
+(the path has no exchange step, so there is no data-path collective); the
+reported time is the max over ranks and the value counts the work of all ranks
+("scaling": "weak").
+
+``--impl reference`` times the float64 CPU oracle on bounded samples of the
+same workload (rank 0 only) and prints the same JSON line with "impl":
+"reference".  The CPU baseline inside the default run does the same once.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s and ms/layer at 32,760 tokens; % of B200 dense BF16 peak"
+
+WORKLOADS = {
+    # name: (B, T latent frames, H latent, W latent, heads, head_dim, description)
+    "480p81_cfg_pair": (2, 21, 60, 104, 40, 128,
+                        "81-frame 832x480 clip, CFG pair: 2 x 21x30x52 = 32,760 tokens, 40 heads x 128"),
+    "720p81": (1, 21, 90, 160, 40, 128, "81-frame 1280x720 clip: 21x45x80 = 75,600 tokens, 40 heads x 128"),
+    "480p17": (1, 5, 60, 104, 12, 128, "17-frame 832x480 clip: 5x30x52 = 7,800 tokens, 12 heads x 128"),
+}
+DEFAULT_WORKLOAD = "480p81_cfg_pair"
+LATENT_C = 16
+PATCH = (1, 2, 2)
+
+
+def workload_dims(name):
+    B, T, H, W, heads, D, desc = WORKLOADS[name]
+    Tg, Hg, Wg = T // PATCH[0], H // PATCH[1], W // PATCH[2]
+    return dict(B=B, T=T, H=H, W=W, heads=heads, D=D, Tg=Tg, Hg=Hg, Wg=Wg, L=Tg * Hg * Wg, HW=Hg * Wg, desc=desc)
+
+
+def step_flops(d):
+    """Algorithmic FLOPs of one step: 4*Lq*Lk*D per (batch, head) for full
+    attention, the time pass (HW sites x T^2) and the space pass (T frames x HW^2)."""
+    B, H, D, L, T, HW = d["B"], d["heads"], d["D"], d["L"], d["Tg"], d["HW"]
+    full = 4 * B * H * L * L * D
+    tpass = 4 * B * H * D * HW * T * T
+    spass = 4 * B * H * D * T * HW * HW
+    return full, tpass, spass
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash():
+    """Hash of the attention kernel's sources: a stored ncu traffic figure is used
+    only while it still describes the kernel that runs."""
+    h = hashlib.sha256()
+    for f in ("attn_tcgen05.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "spacetime_attention_vdit_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload):
+    """DRAM bytes per launch of the full-attention kernel from a committed ncu
+    summary, or None when absent or taken on other kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_full_traffic.json")) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                             parts[5], parts[6], parts[7], parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(d, budget_s, seed=0):
+    """Time the float64 oracle on a bounded sample of the step: query rows of full
+    attention of one (batch, head), plus proportional rows of the space pass.
+    Returns (FLOPs done, seconds, description)."""
+    import synthetic
+    from oracle import reference as ref
+
+    L, D, T, HW = d["L"], d["D"], d["Tg"], d["HW"]
+    q, k, v = synthetic.qkv_bf16(1, L, 1, D, seed=seed)
+    qf, kf, vf = (synthetic.bf16_bits_to_f64(x) for x in (q, k, v))
+    rows = 64
+    flops = 0
+    t0 = time.perf_counter()
+    done_rows = 0
+    while True:
+        sel = synthetic.sample_rows(L, rows, seed=seed + done_rows)
+        ref.attention(qf, kf, vf, rows=sel)
+        ref.divided_space_rows(qf, kf, vf, T, HW, sel)
+        ref.divided_time_rows(qf, kf, vf, T, HW, sel)
+        flops += 4 * rows * L * D + 4 * rows * HW * D + 4 * rows * T * D
+        done_rows += rows
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+        rows = min(4096, rows * 2)
+    return flops, el, f"{done_rows} query rows of one (batch, head): full attention over all {L} keys, " \
+                      f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, d):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    per_step_budget = max(1.0, min(20.0, 150.0 / max(1, steps + warmup)))
+    for _ in range(warmup):
+        oracle_sample(d, per_step_budget / 4)
+    tot_f, tot_s, desc = 0, 0.0, ""
+    for _ in range(steps):
+        f, s, desc = oracle_sample(d, per_step_budget)
+        tot_f += f
+        tot_s += s
+    val = tot_f / tot_s / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * tot_s / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "description": d["desc"], "batch": d["B"], "tokens": d["L"],
+                       "heads": d["heads"], "head_dim": d["D"]},
+            "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s", "cores": cpu_cores(),
+                             "sample": f"per step: {desc}"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    d = workload_dims(args.workload)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.impl == "reference":
+        return run_reference(args, d)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import spacetime_attention_vdit_b200 as vd
+    import synthetic
+
+    B, L, Hh, D, Tg, HW = d["B"], d["L"], d["heads"], d["D"], d["Tg"], d["HW"]
+    grid = (d["Tg"], d["Hg"], d["Wg"])
+    seed = 1000 * rank  # every rank its own clip pair
+    lat_h = torch.from_numpy(synthetic.latent_f32(B, LATENT_C, d["T"], d["H"], d["W"], seed=seed)).pin_memory()
+    qb, kb, vb = synthetic.qkv_bf16(B, L, Hh, D, seed=seed)
+
+    def pinned_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    q_h, k_h, v_h = pinned_bf16(qb), pinned_bf16(kb), pinned_bf16(vb)
+    del qb, kb, vb
+    lat = lat_h.to(dev)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    tok = torch.empty((B, L, LATENT_C * PATCH[0] * PATCH[1] * PATCH[2]), dtype=torch.float32, device=dev)
+    qr, kr = torch.empty_like(q), torch.empty_like(k)
+    o_full, o_time, o_space = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    names = ("patchify", "rope", "attn_full", "attn_time", "attn_space")
+    launches_per_step = len(names)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        vd.patchify_3d(lat, PATCH, out=tok)
+        if ev is not None:
+            ev[1].record(stream)
+        vd.rope_3d(q, k, grid, q_out=qr, k_out=kr)
+        if ev is not None:
+            ev[2].record(stream)
+        vd.attn_full(qr, kr, v, out=o_full)
+        if ev is not None:
+            ev[3].record(stream)
+        vd.attn_divided_time(qr, kr, v, Tg, HW, out=o_time)
+        if ev is not None:
+            ev[4].record(stream)
+        vd.attn_divided_space(qr, kr, v, Tg, HW, out=o_space)
+        if ev is not None:
+            ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    rc, flags = vd.device_status()
+    if rc != 0:
+        raise RuntimeError(f"kernel watchdog tripped during warm-up: flags {flags:#x}")
+
+    # ---- device-resident timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        barrier()
+    clocks = clk.summary()
+    ms_local = start.elapsed_time(stop)
+    ms = max_over_ranks(ms_local)
+    per_row = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(names)}
+    rc, flags = vd.device_status()
+    if rc != 0:
+        raise RuntimeError(f"kernel watchdog tripped in the timed region: flags {flags:#x}")
+
+    full_f, time_f, space_f = step_flops(d)
+    flops_step = full_f + time_f + space_f
+    value = world * flops_step * args.steps / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (tok, o_full, o_time, o_space)]
+        h2d = sum(t.numel() * t.element_size() for t in (lat_h, q_h, k_h, v_h))
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+        def e2e_step():
+            lat.copy_(lat_h, non_blocking=True)
+            q.copy_(q_h, non_blocking=True)
+            k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            step()
+            for hbuf, dbuf in zip(outs_h, (tok, o_full, o_time, o_space)):
+                hbuf.copy_(dbuf, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        e_steps = max(2, min(args.steps, 5))
+        barrier()
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        t2.record(stream)
+        barrier()
+        e_ms = max_over_ranks(s2.elapsed_time(t2))
+        e2e = {"value": world * flops_step * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms / e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": e_steps}
+
+    # ---- roofline of the dominant kernel (full attention)
+    peaks, peaks_kind = measured_peaks()
+    full_ms = per_row["attn_full"]
+    achieved = full_f / (full_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_tcgen05_kernel<128>", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": stored_traffic(args.workload),
+                "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside a long step)",
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "flops_per_launch": full_f, "avg_launch_ms": full_ms}
+
+    hbm = peaks["hbm_gbs"]
+    tok_bytes = tok.numel() * 4
+    row_bytes = {
+        "patchify": lat.numel() * 4 + tok_bytes,
+        "rope": 4 * q.numel() * 2,
+        "attn_time": 4 * q.numel() * 2,
+    }
+    rows = {}
+    for n in names:
+        r = {"ms": per_row[n]}
+        if n in row_bytes:
+            r["gb_s"] = row_bytes[n] / (per_row[n] * 1e-3) / 1e9
+            r["frac_hbm"] = r["gb_s"] / hbm
+        if n == "attn_full":
+            r["tflops"] = achieved
+        if n == "attn_space":
+            r["tflops"] = space_f / (per_row[n] * 1e-3) / 1e12
+        rows[n] = r
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, s, desc = oracle_sample(d, 15.0)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": desc + f"; {s:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "description": d["desc"], "batch": d["B"],
+                           "tokens": L, "heads": Hh, "head_dim": D, "grid": list(grid), "patch": list(PATCH),
+                           "latent": [d["B"], LATENT_C, d["T"], d["H"], d["W"]],
+                           "step": "patchify + rope + full attention + time pass + space pass",
+                           "flops_per_step_per_gpu": flops_step,
+                           "l2": "inputs larger than L2: %.2f GB of Q/K/V per step" % (3 * q.numel() * 2 / 1e9),
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+                "frac_of_nominal_dense_bf16": achieved / 2250.0}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

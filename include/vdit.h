@@ -1,0 +1,191 @@
+/*
+ * vdit.h - C ABI of libvdit.so: spacetime self-attention over video-DiT latent
+ * tokens on NVIDIA B200 (sm_100a).
+ *
+ * The hot path the library runs, in the order a video diffusion transformer
+ * meets it:
+ *
+ *   latent clip [N, C, T, H, W]
+ *     -> vdit_patchify_3d        cut into (pt, ph, pw) spacetime bricks, one token each
+ *     -> (projection to per-head Q, K, V: done by the caller)
+ *     -> vdit_rope_3d            factorised 3D rotary positions on Q and K
+ *     -> vdit_attn_full          full 3D self-attention over all T*H'*W' tokens
+ *        or
+ *        vdit_attn_divided_time  attention over the T tokens at each spatial site
+ *        vdit_attn_divided_space attention over the H'*W' tokens of each frame
+ *
+ * Sources (page title, section):
+ *   [towardsai]  "How AI Generates Video: Inside Sora and Wan2.1 on a Real GPU",
+ *                sections 4 (spacetime tubes, 3D factorized RoPE), 5 (full 3D
+ *                self-attention) and 7 (the [7800 x 7800] matrix, token order).
+ *   [cheatsheet] "Video and 3D Generation" (aiengineeringfromscratch.com):
+ *                "Formulas and numbers" (video tokens, divided attention),
+ *                "Tiny video DiT" (Conv3d patchify, time pass then space pass),
+ *                "Troubleshooting" (the rope_3d split rule).
+ *   [aicassindra] "Video Diffusion Models, in depth": "Step 2: patchify into
+ *                spacetime tokens", "Step 3: the diffusion transformer" (tiled
+ *                attention whose scores never leave the chip).
+ *   [signal3d]   "Video as a 3D signal": "Patches and attention" (full 3-D
+ *                against the factorised form).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller.  The library
+ *    allocates no memory, frees none and never synchronises; it only enqueues
+ *    kernels on `stream` (a cudaStream_t; NULL means the legacy default stream)
+ *    and returns.  Calls are asynchronous: data must stay valid until the
+ *    stream has run them.
+ *  - Token order is time-major, then rows, then columns: token (t', h, w) of a
+ *    (Tg, Hg, Wg) grid sits at position t'*Hg*Wg + h*Wg + w [towardsai s.7].
+ *  - Q, K, V and O are bfloat16, laid out [B, L, heads, head_dim] (token-major,
+ *    heads interleaved: the unpermuted output of a [B, L, heads*head_dim]
+ *    projection), contiguous, 16-byte aligned.  Arithmetic is float32.
+ *  - head_dim must be 32, 64 or 128 for attention (VDIT_ERR_UNSUPPORTED
+ *    otherwise).
+ *  - `scale` <= 0 selects 1/sqrt(head_dim) [towardsai s.7].
+ *  - `lse` may be NULL.  When given it receives float32 [B, heads, L] natural-log
+ *    log-sum-exp of each query row's scaled logits, indexed by the token's own
+ *    position in the sequence.
+ *  - Host-detectable errors (NULL pointers, bad sizes, misalignment,
+ *    unsupported head_dim) return before anything is launched.  A failed
+ *    launch returns VDIT_ERR_CUDA.  Faults during execution surface on the
+ *    caller's stream, as for any CUDA kernel.
+ *  - Every wait inside a kernel is bounded.  A wait that runs out records a
+ *    flag that vdit_device_status() reports (VDIT_ERR_TIMEOUT); until the flag
+ *    is cleared, later launches exit at once instead of computing.
+ */
+#ifndef VDIT_H
+#define VDIT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* vdit_stream_t;
+
+/* Status codes returned by every call. */
+enum vdit_status {
+  VDIT_OK = 0,
+  VDIT_ERR_NULL = 1,        /* a required pointer is NULL                       */
+  VDIT_ERR_SHAPE = 2,       /* a size is non-positive, inconsistent or too big  */
+  VDIT_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                 */
+  VDIT_ERR_UNSUPPORTED = 4, /* valid input this build does not handle           */
+  VDIT_ERR_CUDA = 5,        /* the CUDA runtime reported an error               */
+  VDIT_ERR_TIMEOUT = 6      /* a kernel's bounded wait ran out (device status)  */
+};
+
+/* Element types of the patchify call. */
+enum vdit_dtype { VDIT_F32 = 0, VDIT_BF16 = 1 };
+
+/*
+ * vdit_patchify_3d - spacetime patchify [towardsai s.4; cheatsheet "Tiny video
+ * DiT": a Conv3d whose stride equals its kernel; aicassindra Step 2].
+ *
+ *   tokens[n, (t'*Hg + h')*Wg + w', ((c*pt + dt)*ph + dh)*pw + dw]
+ *       = latent[n, c, t'*pt + dt, h'*ph + dh, w'*pw + dw]
+ *
+ * with (Tg, Hg, Wg) = (T/pt, H/ph, W/pw) floored: voxels past the last whole
+ * brick are not read.  latent: [N, C, T, H, W] contiguous; tokens:
+ * [N, Tg*Hg*Wg, C*pt*ph*pw] contiguous.  dtype VDIT_F32 or VDIT_BF16 for both;
+ * values are copied bit for bit.  Pointers need only the element alignment;
+ * 16-byte alignment enables vector access.  Errors: VDIT_ERR_NULL,
+ * VDIT_ERR_SHAPE (a non-positive size, a grid extent of 0, or more than 2^31
+ * tokens), VDIT_ERR_UNSUPPORTED (dtype), VDIT_ERR_CUDA.
+ */
+int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
+                     int N, int C, int T, int H, int W,
+                     int pt, int ph, int pw, vdit_stream_t stream);
+
+/*
+ * vdit_rope_3d - factorised 3D rotary position embedding [towardsai s.4].
+ *
+ * Q and K are [B, L, heads, head_dim] bfloat16 with L = Tg*Hg*Wg.  Each head
+ * vector is split into a time segment of d_t dims, then d_h, then d_w
+ * (d_t + d_h + d_w = head_dim, each even; (44, 42, 42) for head_dim 128).
+ * Pair i of a segment of width d (elements 2i and 2i+1 of the segment) turns by
+ * the angle pos * theta^(-2i/d), pos being the token's t', h or w on the patch
+ * grid:
+ *     out[2i]   = x[2i]*cos(a) - x[2i+1]*sin(a)
+ *     out[2i+1] = x[2i]*sin(a) + x[2i+1]*cos(a)
+ * Angles are formed in float64 and their cosines and sines rounded once to
+ * float32, as the page's snippet does; the rotation runs in float32 with each
+ * product and sum rounded separately, and the result is rounded to bfloat16
+ * (nearest even).  V is not rotated.  q_out/k_out may equal q_in/k_in (in
+ * place); otherwise the buffers must not overlap.  Errors: VDIT_ERR_NULL,
+ * VDIT_ERR_SHAPE (the split does not add up to head_dim or has an odd or
+ * negative part - the page's rope_3d ValueError; non-positive sizes),
+ * VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED (head_dim not a multiple of 8),
+ * VDIT_ERR_CUDA.
+ */
+int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                 int B, int Tg, int Hg, int Wg, int heads, int head_dim,
+                 int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
+
+/*
+ * vdit_attn_full - full 3D self-attention [towardsai s.5: every token attends
+ * to all tokens; aicassindra Step 3: tiled, the L x L scores never reach HBM].
+ *
+ *   O[b, i, h, :] = sum_j softmax_j(scale * Q[b,i,h,:] . K[b,j,h,:]) V[b, j, h, :]
+ *
+ * over all L tokens, non-causal, no mask.  q, k, v, o: [B, L, heads, head_dim];
+ * lse: NULL or [B, heads, L].  o must not overlap q, k or v.  Runs on the
+ * tensor cores (bf16 inputs, float32 accumulation); P is rounded to bfloat16
+ * before the P.V product; O is rounded to bfloat16 (nearest even).
+ * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED,
+ * VDIT_ERR_CUDA.
+ */
+int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int L, int heads, int head_dim, float scale,
+                   vdit_stream_t stream);
+
+/*
+ * vdit_attn_divided_time - the time pass of divided attention [cheatsheet
+ * "Tiny video DiT" and "Divided attention"; signal3d "Patches and attention"].
+ *
+ * The sequence holds L = T*HW tokens (T frames of HW sites, frame-major).  For
+ * each batch b, site s and head h, attention runs over the T tokens
+ * {t*HW + s : t < T}; it equals full attention restricted to pairs at the same
+ * site.  Buffers as for vdit_attn_full (read and written in place of the
+ * tokens; nothing is transposed).  lse: NULL or [B, heads, T*HW].
+ * Errors as for vdit_attn_full.
+ */
+int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int T, int HW, int heads, int head_dim, float scale,
+                           vdit_stream_t stream);
+
+/*
+ * vdit_attn_divided_space - the space pass of divided attention (same sources).
+ *
+ * For each batch b, frame t and head h, attention runs over the HW tokens of
+ * frame t, positions [t*HW, (t+1)*HW); it equals full attention restricted to
+ * pairs in the same frame.  Buffers and errors as for
+ * vdit_attn_divided_time; lse: NULL or [B, heads, T*HW].
+ */
+int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int T, int HW, int heads, int head_dim, float scale,
+                            vdit_stream_t stream);
+
+/* Text for a status code (static storage; never NULL). */
+const char* vdit_status_string(int status);
+
+/*
+ * vdit_device_status - report and clear the watchdog flags that kernels set
+ * when a bounded wait runs out.  Synchronises the current device first (the
+ * one call here that does).  *flags (may be NULL) receives the raw bit set:
+ * bit 0 any timeout, bits 8.. the wait site.  Returns VDIT_OK when no flag was
+ * set, VDIT_ERR_TIMEOUT when one was, VDIT_ERR_CUDA if the device reported an
+ * error.
+ */
+int vdit_device_status(unsigned int* flags);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int vdit_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDIT_H */

@@ -91,14 +91,15 @@ def rope_inv_freq(d_axis: int, theta: float = 10000.0) -> np.ndarray:
     return 1.0 / (theta ** (j / d_axis))
 
 
-def rope_tables(grid, split, theta: float = 10000.0):
+def rope_tables(grid, split, theta: float = 10000.0, tokens=None):
     """Per-token angles for every pair of the head: array [L, D/2] float64.
 
     Pair i < d_t/2 turns by t'*f_t[i]; the next d_h/2 pairs by h*f_h[i]; the last
-    d_w/2 pairs by w*f_w[i]; positions are patch-grid indices."""
+    d_w/2 pairs by w*f_w[i]; positions are patch-grid indices.  ``tokens``
+    restricts the rows to those sequence positions."""
     Tg, Hg, Wg = grid
     L = Tg * Hg * Wg
-    idx = np.arange(L)
+    idx = np.arange(L) if tokens is None else np.asarray(tokens)
     t, h, w = grid_position(idx, grid)
     parts = []
     for pos, d in zip((t, h, w), split):
@@ -106,16 +107,17 @@ def rope_tables(grid, split, theta: float = 10000.0):
     return np.concatenate(parts, axis=1)
 
 
-def rope_3d(x: np.ndarray, grid, split, theta: float = 10000.0) -> np.ndarray:
+def rope_3d(x: np.ndarray, grid, split, theta: float = 10000.0, tokens=None) -> np.ndarray:
     """Rotate Q or K ``[B, L, heads, D]`` in float64.
 
     For pair p = (x[2p], x[2p+1]) with angle a: (x0*cos a - x1*sin a,
-    x0*sin a + x1*cos a), i.e. the complex product (x0 + i x1) * e^{ia}."""
+    x0*sin a + x1*cos a), i.e. the complex product (x0 + i x1) * e^{ia}.
+    ``tokens`` gives the sequence positions of x's rows when x holds a subset."""
     B, L, Hh, D = x.shape
     check_split(D, split)
-    if L != grid[0] * grid[1] * grid[2]:
+    if tokens is None and L != grid[0] * grid[1] * grid[2]:
         raise ValueError("sequence length does not match the token grid")
-    ang = rope_tables(grid, split, theta)            # [L, D/2]
+    ang = rope_tables(grid, split, theta, tokens)    # [L, D/2]
     c = np.cos(ang)[None, :, None, :]
     s = np.sin(ang)[None, :, None, :]
     x = np.asarray(x, dtype=np.float64)
@@ -127,7 +129,7 @@ def rope_3d(x: np.ndarray, grid, split, theta: float = 10000.0) -> np.ndarray:
     return out
 
 
-def rope_3d_fp32(x32: np.ndarray, grid, split, theta: float = 10000.0) -> np.ndarray:
+def rope_3d_fp32(x32: np.ndarray, grid, split, theta: float = 10000.0, tokens=None) -> np.ndarray:
     """The same rotation at the towardsai snippet's own precision.
 
     The snippet builds angles in float64 and stores the phasors as complex64,
@@ -138,7 +140,7 @@ def rope_3d_fp32(x32: np.ndarray, grid, split, theta: float = 10000.0) -> np.nda
     """
     B, L, Hh, D = x32.shape
     check_split(D, split)
-    ang = rope_tables(grid, split, theta)
+    ang = rope_tables(grid, split, theta, tokens)
     c = np.cos(ang).astype(np.float32)[None, :, None, :]
     s = np.sin(ang).astype(np.float32)[None, :, None, :]
     x32 = np.asarray(x32, dtype=np.float32)
@@ -271,6 +273,48 @@ def divided_space(q, k, v, T: int, HW: int, scale=None, frames=None):
     o, lse = attention(to_seq(q), to_seq(k), to_seq(v), scale)
     o = o.reshape(B, fr.size * HW, Hh, -1)
     lse = lse.reshape(B, fr.size, Hh, HW).transpose(0, 2, 1, 3).reshape(B, Hh, fr.size * HW)
+    return o, lse
+
+
+def divided_time_rows(q, k, v, T: int, HW: int, rows, scale=None):
+    """Selected query rows of the time pass: the row at sequence position r
+    attends over the T tokens {t*HW + r % HW} of its site.  q, k, v
+    [B, T*HW, H, D]; returns (o [B, R, H, D], lse [B, H, R])."""
+    rows = np.asarray(rows)
+    B, L, Hh, D = np.shape(q)
+    if scale is None or scale <= 0:
+        scale = default_scale(D)
+    keys = np.arange(T)[None, :] * HW + (rows % HW)[:, None]      # [R, T]
+    o = np.empty((B, rows.size, Hh, np.shape(v)[-1]))
+    lse = np.empty((B, Hh, rows.size))
+    for b in range(B):
+        for h in range(Hh):
+            qr = np.asarray(q[b, rows, h, :], dtype=np.float64)           # [R, D]
+            kr = np.asarray(k[b, keys, h, :], dtype=np.float64)           # [R, T, D]
+            vr = np.asarray(v[b, keys, h, :], dtype=np.float64)
+            s = np.einsum("rd,rtd->rt", qr, kr) * scale
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            l = p.sum(axis=1, keepdims=True)
+            o[b, :, h, :] = np.einsum("rt,rtd->rd", p, vr) / l
+            lse[b, h] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def divided_space_rows(q, k, v, T: int, HW: int, rows, scale=None):
+    """Selected query rows of the space pass: the row at position r attends over
+    the HW tokens of its frame r // HW.  Returns (o [B, R, H, D], lse [B, H, R])."""
+    rows = np.asarray(rows)
+    B, L, Hh, D = np.shape(q)
+    o = np.empty((B, rows.size, Hh, np.shape(v)[-1]))
+    lse = np.empty((B, Hh, rows.size))
+    frame = rows // HW
+    for f in np.unique(frame):
+        sel = np.nonzero(frame == f)[0]
+        sl = slice(f * HW, (f + 1) * HW)
+        of, lf = attention(q[:, sl], k[:, sl], v[:, sl], scale, rows=rows[sel] - f * HW)
+        o[:, sel] = of
+        lse[:, :, sel] = lf
     return o, lse
 
 

@@ -1,0 +1,213 @@
+"""Python binding of libvdit.so: spacetime self-attention over video-DiT tokens.
+
+A thin ctypes layer: it checks that tensors are CUDA, contiguous and of the
+right dtype and shape, passes their device pointers, sizes and the current
+CUDA stream to the C ABI declared in ``include/vdit.h``, and raises
+:class:`VditError` on a nonzero status.  Every step of the path runs in the
+library's kernels; there is no fallback.  PyTorch is used only for device
+memory and streams (outputs are allocated with ``torch.empty`` when the caller
+passes none).
+
+Calls (see ``include/vdit.h`` for the exact definitions and sources):
+
+* :func:`patchify_3d`         latent [N, C, T, H, W] -> tokens [N, L, C*pt*ph*pw]
+* :func:`rope_3d`             3D rotary positions on Q and K [B, L, heads, D]
+* :func:`attn_full`           full 3D self-attention
+* :func:`attn_divided_time`   attention over the T tokens of each spatial site
+* :func:`attn_divided_space`  attention over the HW tokens of each frame
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["VditError", "lib", "patchify_3d", "rope_3d", "attn_full", "attn_divided_time",
+           "attn_divided_space", "device_status", "status_string", "default_split", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "VDIT_OK", 1: "VDIT_ERR_NULL", 2: "VDIT_ERR_SHAPE", 3: "VDIT_ERR_ALIGN",
+           4: "VDIT_ERR_UNSUPPORTED", 5: "VDIT_ERR_CUDA", 6: "VDIT_ERR_TIMEOUT"}
+
+
+class VditError(RuntimeError):
+    """A libvdit call returned a nonzero status."""
+
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call}: {_STATUS.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_SIGNATURES = {
+    "vdit_patchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
+    "vdit_rope_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
+    "vdit_attn_full": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P],
+    "vdit_attn_divided_time": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
+    "vdit_attn_divided_space": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
+    "vdit_device_status": [ctypes.POINTER(ctypes.c_uint)],
+    "vdit_version": [],
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if libvdit.so has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libvdit.so not built at {LIB_PATH}: run "
+                              "`python -m spacetime_attention_vdit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.vdit_status_string.argtypes = [ctypes.c_int]
+        L.vdit_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().vdit_status_string(int(status)).decode()
+
+
+def _check(call: str, rc: int) -> None:
+    if rc != 0:
+        raise VditError(call, rc)
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def default_split(head_dim: int):
+    """(44, 42, 42) for head_dim 128: time takes the remainder, height and width
+    2*floor(head_dim/6) each."""
+    s = 2 * (head_dim // 6)
+    return (head_dim - 2 * s, s, s)
+
+
+def patchify_3d(latent: torch.Tensor, patch=(1, 2, 2), out: torch.Tensor | None = None, stream=None):
+    """Cut ``latent`` [N, C, T, H, W] (float32 or bfloat16) into (pt, ph, pw) bricks;
+    returns tokens [N, Tg*Hg*Wg, C*pt*ph*pw] of the same dtype."""
+    if latent.dim() != 5:
+        raise ValueError("latent must be [N, C, T, H, W]")
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(latent.dtype)
+    if dt is None:
+        raise ValueError("latent must be float32 or bfloat16")
+    N, C, T, H, W = latent.shape
+    pt, ph, pw = patch
+    L = (T // pt) * (H // ph) * (W // pw)
+    F = C * pt * ph * pw
+    if out is None:
+        out = torch.empty((N, L, F), dtype=latent.dtype, device=latent.device)
+    elif tuple(out.shape) != (N, L, F):
+        raise ValueError(f"out must be {(N, L, F)}")
+    _check("vdit_patchify_3d", lib().vdit_patchify_3d(
+        _dev(latent, "latent"), _dev(out, "out", latent.dtype), dt, N, C, T, H, W, pt, ph, pw, _stream(stream)))
+    return out
+
+
+def rope_3d(q: torch.Tensor, k: torch.Tensor, grid, split=None, theta: float = 10000.0,
+            q_out: torch.Tensor | None = None, k_out: torch.Tensor | None = None, inplace: bool = False,
+            stream=None):
+    """Rotate Q and K ([B, L, heads, D] bfloat16, L = Tg*Hg*Wg) by their 3D grid
+    positions.  ``split`` = (d_t, d_h, d_w), default :func:`default_split`.
+    Returns (q_out, k_out); with ``inplace`` the inputs are overwritten."""
+    if q.dim() != 4 or q.shape != k.shape:
+        raise ValueError("q and k must both be [B, L, heads, head_dim]")
+    B, L, Hh, D = q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != L:
+        raise ValueError("grid does not match the sequence length")
+    d_t, d_h, d_w = default_split(D) if split is None else split
+    if inplace:
+        q_out, k_out = q, k
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    _check("vdit_rope_3d", lib().vdit_rope_3d(
+        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
+        _dev(k_out, "k_out", torch.bfloat16), B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
+    return q_out, k_out
+
+
+def _attn_io(q, k, v, out, lse):
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k and v must all be [B, L, heads, head_dim]")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n, torch.bfloat16)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    B, L, Hh, D = q.shape
+    lse_t = None
+    if lse is True:
+        lse_t = torch.empty((B, Hh, L), dtype=torch.float32, device=q.device)
+    elif isinstance(lse, torch.Tensor):
+        if tuple(lse.shape) != (B, Hh, L):
+            raise ValueError(f"lse must be {(B, Hh, L)}")
+        lse_t = lse
+    lse_p = None if lse_t is None else _dev(lse_t, "lse", torch.float32)
+    return out, lse_t, lse_p
+
+
+def attn_full(q, k, v, out=None, lse=None, scale: float = 0.0, stream=None):
+    """O = softmax(scale Q K^T) V over all L tokens of each (batch, head).
+    ``lse=True`` also returns the float32 [B, heads, L] log-sum-exp."""
+    out, lse_t, lse_p = _attn_io(q, k, v, out, lse)
+    B, L, Hh, D = q.shape
+    _check("vdit_attn_full", lib().vdit_attn_full(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, L, Hh, D,
+        float(scale), _stream(stream)))
+    return out if lse_t is None else (out, lse_t)
+
+
+def _divided(name, q, k, v, T, HW, out, lse, scale, stream):
+    out, lse_t, lse_p = _attn_io(q, k, v, out, lse)
+    B, L, Hh, D = q.shape
+    if T * HW != L:
+        raise ValueError("L must equal T * HW")
+    _check(name, getattr(lib(), name)(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, T, HW, Hh, D,
+        float(scale), _stream(stream)))
+    return out if lse_t is None else (out, lse_t)
+
+
+def attn_divided_time(q, k, v, T: int, HW: int, out=None, lse=None, scale: float = 0.0, stream=None):
+    """Time pass: attention over the T tokens {t*HW + s} of each site s."""
+    return _divided("vdit_attn_divided_time", q, k, v, T, HW, out, lse, scale, stream)
+
+
+def attn_divided_space(q, k, v, T: int, HW: int, out=None, lse=None, scale: float = 0.0, stream=None):
+    """Space pass: attention over the HW tokens of each frame t."""
+    return _divided("vdit_attn_divided_space", q, k, v, T, HW, out, lse, scale, stream)
+
+
+def device_status():
+    """(status, flags) of the kernels' bounded waits since the last call; synchronises."""
+    flags = ctypes.c_uint(0)
+    rc = lib().vdit_device_status(ctypes.byref(flags))
+    return rc, flags.value

@@ -1,0 +1,185 @@
+// patchify_rope.cuh - the two bandwidth-bound steps of the path.
+//
+// Spacetime patchify ("How AI Generates Video: Inside Sora and Wan2.1 on a Real
+// GPU", section 4; "Video and 3D Generation" cheatsheet, "Tiny video DiT": a
+// Conv3d whose stride equals its kernel) is a pure permutation of the latent
+// clip.  Factorised 3D RoPE (same article, section 4) rotates adjacent pairs of
+// every Q and K head vector by angles set by the token's (t', h, w).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace vdit {
+
+// ---------------------------------------------------------------------------
+// Patchify
+// ---------------------------------------------------------------------------
+//
+// One CTA owns a run of WC bricks that share (n, t', h') - consecutive tokens,
+// so its output is one contiguous span of WC*F elements (F = C*pt*ph*pw).  The
+// CTA first copies the C*pt*ph latent rows those bricks cover (each a
+// contiguous run of WC*pw elements along W) into shared memory with coalesced
+// loads, then writes the output span in order with coalesced stores, reading
+// each element's source from shared memory by the brick index formula.
+
+struct PatchifyShape {
+  int N, C, T, H, W, pt, ph, pw;
+  int Tg, Hg, Wg;   // patch grid (floored)
+  int F;            // features per token
+  int WC;           // bricks per CTA along w'
+  int n_wchunks;    // ceil(Wg / WC)
+};
+
+template <typename E>
+__global__ void __launch_bounds__(256) patchify3d_kernel(const E* __restrict__ latent, E* __restrict__ tokens,
+                                                         PatchifyShape s) {
+  E* rows = reinterpret_cast<E*>(dyn_smem);
+  if (watchdog_tripped()) return;
+
+  const int rowlen = s.WC * s.pw;                 // elements per staged row
+  const int nrows = s.C * s.pt * s.ph;
+
+  for (long long job = blockIdx.x; job < (long long)s.N * s.Tg * s.Hg * s.n_wchunks; job += gridDim.x) {
+    const int wc = (int)(job % s.n_wchunks);
+    long long r = job / s.n_wchunks;
+    const int hq = (int)(r % s.Hg);
+    r /= s.Hg;
+    const int tq = (int)(r % s.Tg);
+    const int n = (int)(r / s.Tg);
+    const int w0 = wc * s.WC;
+    const int nb = min(s.WC, s.Wg - w0);          // bricks in this chunk
+    const int len = nb * s.pw;                    // valid elements per staged row
+
+    // stage latent rows (c, dt, dh) -> rows[((c*pt + dt)*ph + dh) * rowlen + x]
+    for (int i = threadIdx.x; i < nrows * len; i += blockDim.x) {
+      const int row = i / len, x = i - row * len;
+      const int dh = row % s.ph;
+      const int dt = (row / s.ph) % s.pt;
+      const int c = row / (s.ph * s.pt);
+      const long long src =
+          ((((long long)n * s.C + c) * s.T + (tq * s.pt + dt)) * s.H + (hq * s.ph + dh)) * s.W + (long long)w0 * s.pw + x;
+      rows[row * rowlen + x] = latent[src];
+    }
+    __syncthreads();
+
+    // write the contiguous output span of nb tokens
+    const long long tok0 = ((long long)n * s.Tg + tq) * s.Hg * s.Wg + (long long)hq * s.Wg + w0;
+    E* out = tokens + tok0 * s.F;
+    const int ppw = s.ph * s.pw, pppw = s.pt * ppw;
+    for (int i = threadIdx.x; i < nb * s.F; i += blockDim.x) {
+      const int b = i / s.F, f = i - b * s.F;
+      const int c = f / pppw;
+      const int rem = f - c * pppw;
+      const int dt = rem / ppw;
+      const int dh = (rem / s.pw) % s.ph;
+      const int dw = rem % s.pw;
+      out[i] = rows[((c * s.pt + dt) * s.ph + dh) * rowlen + b * s.pw + dw];
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3D RoPE
+// ---------------------------------------------------------------------------
+//
+// A CTA handles kRopeTokens tokens per iteration (grid-stride over tokens).
+// For those tokens it first builds the (cos, sin) of every pair in shared
+// memory: angle = pos * inv_freq in float64, cos and sin in float64, each
+// rounded once to float32 (the snippet's complex64 cache).  inv_freq[p] =
+// 1 / theta^(2i/d) for pair i of its axis segment is built once per CTA.  Then
+// all heads of Q and K for those tokens stream through 16-byte vectors (four
+// pairs each); each pair is rotated with separately rounded float32 products
+// and sums and stored as bfloat16, round to nearest even.
+
+constexpr int kRopeThreads = 256;
+constexpr int kRopeTokens = 4;
+constexpr int kRopeMaxPairs = 128;  // head_dim <= 256
+constexpr int kRopeBatch = 4;       // 16-byte loads in flight per thread
+
+struct RopeShape {
+  long long ntok;     // B * L
+  int L, Hg, Wg;      // tokens per sequence, grid rows and columns
+  int heads, D;       // head count, head width
+  int pt_end, ph_end; // pair index where the h segment starts, and the w segment
+  int d_t, d_h, d_w;
+};
+
+__global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat16* q_in, const __nv_bfloat16* k_in,
+                                                              __nv_bfloat16* q_out, __nv_bfloat16* k_out,
+                                                              RopeShape s, double theta) {
+  __shared__ double inv_freq[kRopeMaxPairs];
+  __shared__ float2 cs[kRopeTokens][kRopeMaxPairs];
+  if (watchdog_tripped()) return;
+
+  const int P = s.D / 2;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    int i, d;
+    if (p < s.pt_end) { i = p; d = s.d_t; }
+    else if (p < s.ph_end) { i = p - s.pt_end; d = s.d_h; }
+    else { i = p - s.ph_end; d = s.d_w; }
+    inv_freq[p] = 1.0 / pow(theta, (double)(2 * i) / (double)d);
+  }
+  __syncthreads();
+
+  const int vec_per_head = s.D / 8;                      // 16-byte vectors (4 pairs) per head
+  const int vec_per_tok = s.heads * vec_per_head;        // per tensor
+  for (long long tok0 = (long long)blockIdx.x * kRopeTokens; tok0 < s.ntok;
+       tok0 += (long long)gridDim.x * kRopeTokens) {
+    const int nt = (int)min((long long)kRopeTokens, s.ntok - tok0);
+    for (int e = threadIdx.x; e < nt * P; e += blockDim.x) {
+      const int j = e / P, p = e - j * P;
+      const int l = (int)((tok0 + j) % s.L);
+      int pos;
+      if (p < s.pt_end) pos = l / (s.Hg * s.Wg);
+      else if (p < s.ph_end) pos = (l / s.Wg) % s.Hg;
+      else pos = l % s.Wg;
+      double sn, cn;
+      sincos((double)pos * inv_freq[p], &sn, &cn);
+      cs[j][p] = make_float2((float)cn, (float)sn);
+    }
+    __syncthreads();
+
+    // Each thread keeps kRopeBatch 16-byte loads in flight before rotating them.
+    // Every vector is read and written by the same thread, so in-place use is safe.
+    const int nvec = nt * vec_per_tok;                   // per tensor
+    for (int e0 = threadIdx.x; e0 < 2 * nvec; e0 += blockDim.x * kRopeBatch) {
+      uint4 v[kRopeBatch];
+#pragma unroll
+      for (int u = 0; u < kRopeBatch; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < 2 * nvec) {
+          const int which = e >= nvec;                   // 0: Q, 1: K
+          const int ee = which ? e - nvec : e;
+          const long long off = tok0 * (long long)vec_per_tok + ee;
+          v[u] = *(reinterpret_cast<const uint4*>(which ? k_in : q_in) + off);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRopeBatch; ++u) {
+        const int e = e0 + u * blockDim.x;
+        if (e < 2 * nvec) {
+          const int which = e >= nvec;
+          const int ee = which ? e - nvec : e;
+          const int j = ee / vec_per_tok;
+          const int p0 = ((ee - j * vec_per_tok) % vec_per_head) * 4;
+          uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[t]);
+            const float x0 = __low2float(pr), x1 = __high2float(pr);
+            const float2 c = cs[j][p0 + t];
+            const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
+            const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
+            w[t] = pack_bf16x2(re, im);
+          }
+          const long long off = tok0 * (long long)vec_per_tok + ee;
+          *(reinterpret_cast<uint4*>(which ? k_out : q_out) + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace vdit

@@ -1,0 +1,328 @@
+// vdit_api.cu - the C ABI of libvdit.so (declared in include/vdit.h).
+//
+// Host side only: argument checks that return before any launch, tensor-map
+// encoding for the TMA loads, grid sizing, and the launches themselves.  One
+// translation unit holds every kernel so that the watchdog flag is a single
+// device symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "vdit.h"
+#include "attn_tcgen05.cuh"
+#include "attn_time_short.cuh"
+#include "patchify_rope.cuh"
+
+namespace {
+
+using namespace vdit;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int last_launch_status() { return cudaGetLastError() == cudaSuccess ? VDIT_OK : VDIT_ERR_CUDA; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Set a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+bool ensure_smem(K kernel, int bytes, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps
+// ---------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 5-D view {head_dim, heads, sites, positions, batches} of a bf16 [.., heads, D]
+// token array; box {DBLK, 1, 1, 128, 1}.  Rows outside the positions extent
+// read as zero.
+bool make_qkv_map(CUtensorMap* map, const void* base, int D, int heads, long long sites, long long positions,
+                  long long batches, long long site_stride_el, long long pos_stride_el, long long batch_stride_el) {
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return false;
+  const int rowb = D * 2 >= 128 ? 128 : D * 2;
+  const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)sites, (cuuint64_t)positions,
+                              (cuuint64_t)batches};
+  const cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)site_stride_el * 2, (cuuint64_t)pos_stride_el * 2,
+                                 (cuuint64_t)batch_stride_el * 2};
+  const cuuint32_t box[5] = {(cuuint32_t)(rowb / 2), 1, 1, 128, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Attention launches
+// ---------------------------------------------------------------------------
+
+template <int D>
+int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq, int L,
+                   int grp, int heads, float scale, cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  static bool smem_done[kMaxDevices] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ensure_smem(attn_fwd_tcgen05_kernel<D>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
+  }
+  // geometry of the 5-D view
+  long long sites, positions, batches, site_stride, pos_stride, batch_stride;
+  const long long tok = (long long)heads * D;      // elements per token
+  if (mode == kTime) {            // sequence = one site across frames
+    sites = grp;
+    positions = L;
+    batches = n_seq / grp;
+    site_stride = tok;
+    pos_stride = tok * grp;
+    batch_stride = tok * grp * L;
+  } else {                        // sequence = a contiguous run of L tokens
+    sites = 1;
+    positions = L;
+    batches = n_seq;
+    site_stride = tok;
+    pos_stride = tok;
+    batch_stride = tok * L;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, q, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride) ||
+      !make_qkv_map(&mk, k, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride) ||
+      !make_qkv_map(&mv, v, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride))
+    return VDIT_ERR_CUDA;
+  AttnParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.n_seq = n_seq;
+  p.L = L;
+  p.heads = heads;
+  p.grp = grp;
+  p.mode = mode;
+  p.n_qtiles = (L + C::BM - 1) / C::BM;
+  p.n_kv = (L + C::BN - 1) / C::BN;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = (long long)n_seq * heads * p.n_qtiles;
+  if (grid > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  attn_fwd_tcgen05_kernel<D><<<(unsigned)grid, 192, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return last_launch_status();
+}
+
+int dispatch_tcgen05(int D, const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq,
+                     int L, int grp, int heads, float scale, cudaStream_t stream) {
+  switch (D) {
+    case 32: return launch_tcgen05<32>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
+    case 64: return launch_tcgen05<64>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
+    case 128: return launch_tcgen05<128>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
+    default: return VDIT_ERR_UNSUPPORTED;
+  }
+}
+
+template <int D, int TP>
+int launch_time_short(const TimeParams& p, cudaStream_t stream) {
+  using C = TimeCfg<D, TP>;
+  static bool smem_done[kMaxDevices] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ensure_smem(attn_time_short_kernel<D, TP>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
+  }
+  const long long units = (long long)p.B * p.HW * p.heads;
+  const long long want = (units + C::WARPS - 1) / C::WARPS;
+  const long long cap = (long long)sm_count() * 8;   // grid-stride beyond this
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  attn_time_short_kernel<D, TP><<<grid, C::WARPS * 32, C::SMEM_BYTES, stream>>>(p);
+  return last_launch_status();
+}
+
+template <int D>
+int dispatch_time_short_tp(const TimeParams& p, cudaStream_t stream) {
+  if (p.T <= 16) return launch_time_short<D, 16>(p, stream);
+  if (p.T <= 32) return launch_time_short<D, 32>(p, stream);
+  return launch_time_short<D, 64>(p, stream);
+}
+
+float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)D); }
+
+int check_attn_args(const void* q, const void* k, const void* v, const void* o, const float* lse, long long B,
+                    long long L, int heads, int D) {
+  if (!q || !k || !v || !o) return VDIT_ERR_NULL;
+  if (B <= 0 || L <= 0 || heads <= 0 || D <= 0) return VDIT_ERR_SHAPE;
+  if (D != 32 && D != 64 && D != 128) return VDIT_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return VDIT_ERR_ALIGN;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return VDIT_ERR_ALIGN;
+  // element offsets stay below 2^62 and tensor-map extents below 2^32
+  if ((double)B * (double)L * (double)heads * (double)D > 4.0e18 || L > 0xffffffffLL || B > 0xffffffffLL)
+    return VDIT_ERR_SHAPE;
+  return VDIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vdit_version(void) { return 10000; }
+
+const char* vdit_status_string(int status) {
+  switch (status) {
+    case VDIT_OK: return "ok";
+    case VDIT_ERR_NULL: return "a required pointer is NULL";
+    case VDIT_ERR_SHAPE: return "a size is non-positive, inconsistent or too large";
+    case VDIT_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case VDIT_ERR_UNSUPPORTED: return "valid input this build does not handle";
+    case VDIT_ERR_CUDA: return "the CUDA runtime reported an error";
+    case VDIT_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    default: return "unknown status";
+  }
+}
+
+int vdit_device_status(unsigned int* flags) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return VDIT_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_watchdog, sizeof(v)) != cudaSuccess) return VDIT_ERR_CUDA;
+  if (flags != nullptr) *flags = v;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_watchdog, &zero, sizeof(zero)) != cudaSuccess) return VDIT_ERR_CUDA;
+    return VDIT_ERR_TIMEOUT;
+  }
+  return VDIT_OK;
+}
+
+int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, int T, int H, int W, int pt, int ph,
+                     int pw, vdit_stream_t stream) {
+  if (!latent || !tokens) return VDIT_ERR_NULL;
+  if (dtype != VDIT_F32 && dtype != VDIT_BF16) return VDIT_ERR_UNSUPPORTED;
+  if (N <= 0 || C <= 0 || T <= 0 || H <= 0 || W <= 0 || pt <= 0 || ph <= 0 || pw <= 0) return VDIT_ERR_SHAPE;
+  PatchifyShape s;
+  s.N = N; s.C = C; s.T = T; s.H = H; s.W = W; s.pt = pt; s.ph = ph; s.pw = pw;
+  s.Tg = T / pt; s.Hg = H / ph; s.Wg = W / pw;
+  if (s.Tg == 0 || s.Hg == 0 || s.Wg == 0) return VDIT_ERR_SHAPE;
+  const long long F = (long long)C * pt * ph * pw;
+  const long long ntok = (long long)N * s.Tg * s.Hg * s.Wg;
+  if (ntok > 0x7fffffffLL || F > 0x7fffffffLL || (double)ntok * (double)F > 4.0e18) return VDIT_ERR_SHAPE;
+  const int esz = dtype == VDIT_F32 ? 4 : 2;
+  const long long brick_bytes = F * esz;
+  constexpr long long kStage = 32 * 1024;          // staged latent rows per CTA
+  if (brick_bytes > kStage) return VDIT_ERR_UNSUPPORTED;
+  s.F = (int)F;
+  s.WC = (int)std::min<long long>(s.Wg, kStage / brick_bytes);
+  s.n_wchunks = (s.Wg + s.WC - 1) / s.WC;
+  const int smem = (int)((long long)C * pt * ph * s.WC * pw * esz);
+  const long long jobs = (long long)N * s.Tg * s.Hg * s.n_wchunks;
+  const long long cap = (long long)sm_count() * 16;
+  const unsigned grid = (unsigned)(jobs < cap ? jobs : cap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == VDIT_F32)
+    patchify3d_kernel<float><<<grid, 256, smem, st>>>(static_cast<const float*>(latent), static_cast<float*>(tokens), s);
+  else
+    patchify3d_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(latent),
+                                                              static_cast<__nv_bfloat16*>(tokens), s);
+  return last_launch_status();
+}
+
+int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, int B, int Tg, int Hg, int Wg,
+                 int heads, int head_dim, int d_t, int d_h, int d_w, float theta, vdit_stream_t stream) {
+  if (!q_in || !k_in || !q_out || !k_out) return VDIT_ERR_NULL;
+  if (B <= 0 || Tg <= 0 || Hg <= 0 || Wg <= 0 || heads <= 0 || head_dim <= 0) return VDIT_ERR_SHAPE;
+  if (d_t < 0 || d_h < 0 || d_w < 0 || (d_t | d_h | d_w) & 1 || d_t + d_h + d_w != head_dim) return VDIT_ERR_SHAPE;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return VDIT_ERR_SHAPE;
+  if (head_dim % 8 != 0 || head_dim / 2 > kRopeMaxPairs) return VDIT_ERR_UNSUPPORTED;
+  if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out)) return VDIT_ERR_ALIGN;
+  const long long L = (long long)Tg * Hg * Wg;
+  if (L > 0x7fffffffLL || (double)B * (double)L * heads * head_dim > 4.0e18) return VDIT_ERR_SHAPE;
+  RopeShape s;
+  s.ntok = (long long)B * L;
+  s.L = (int)L; s.Hg = Hg; s.Wg = Wg;
+  s.heads = heads; s.D = head_dim;
+  s.pt_end = d_t / 2; s.ph_end = (d_t + d_h) / 2;
+  s.d_t = d_t; s.d_h = d_h; s.d_w = d_w;
+  const long long want = (s.ntok + kRopeTokens - 1) / kRopeTokens;
+  const long long cap = (long long)sm_count() * 8;
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  rope3d_kernel<<<grid, kRopeThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(q_in), static_cast<const __nv_bfloat16*>(k_in),
+      static_cast<__nv_bfloat16*>(q_out), static_cast<__nv_bfloat16*>(k_out), s, (double)theta);
+  return last_launch_status();
+}
+
+int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int heads,
+                   int head_dim, float scale, vdit_stream_t stream) {
+  const int rc = check_attn_args(q, k, v, o, lse, B, L, heads, head_dim);
+  if (rc != VDIT_OK) return rc;
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, L, 1, heads, resolve_scale(scale, head_dim),
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int HW,
+                            int heads, int head_dim, float scale, vdit_stream_t stream) {
+  if (T <= 0 || HW <= 0 || B <= 0) return (!q || !k || !v || !o) ? VDIT_ERR_NULL : VDIT_ERR_SHAPE;
+  const int rc = check_attn_args(q, k, v, o, lse, (long long)B * T, HW, heads, head_dim);
+  if (rc != VDIT_OK) return rc;
+  if ((long long)B * T > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B * T, HW, T, heads, resolve_scale(scale, head_dim),
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int HW,
+                           int heads, int head_dim, float scale, vdit_stream_t stream) {
+  if (T <= 0 || HW <= 0 || B <= 0) return (!q || !k || !v || !o) ? VDIT_ERR_NULL : VDIT_ERR_SHAPE;
+  const int rc = check_attn_args(q, k, v, o, lse, (long long)B * HW, T, heads, head_dim);
+  if (rc != VDIT_OK) return rc;
+  if ((long long)B * HW > 0x7fffffffLL || (long long)T * HW > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  const float sc = resolve_scale(scale, head_dim);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T > 64)  // long clips: the tensor-core kernel over a strided view, one sequence per site
+    return dispatch_tcgen05(head_dim, q, k, v, o, lse, kTime, B * HW, T, HW, heads, sc, st);
+  TimeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B; p.T = T; p.HW = HW; p.heads = heads;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  switch (head_dim) {
+    case 32: return dispatch_time_short_tp<32>(p, st);
+    case 64: return dispatch_time_short_tp<64>(p, st);
+    case 128: return dispatch_time_short_tp<128>(p, st);
+    default: return VDIT_ERR_UNSUPPORTED;
+  }
+}
+
+}  // extern "C"

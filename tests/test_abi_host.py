@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/vdit.h declares, and rejects bad arguments with the
+documented status before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from tests.conftest import ROOT
+
+OK, NULL, SHAPE, ALIGN, UNSUP = 0, 1, 2, 3, 4
+FAKE = 0x7f0000000000          # 16-byte aligned, never dereferenced: every call below returns first
+MIS = FAKE + 8                 # 8-byte aligned only
+
+
+@pytest.fixture(scope="module")
+def L():
+    import spacetime_attention_vdit_b200 as v
+    if not os.path.exists(v.LIB_PATH):
+        v_build = __import__("spacetime_attention_vdit_b200.build", fromlist=["build"])
+        v_build.build()
+    return v.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "vdit.h")).read()
+    return sorted(set(re.findall(r"^(?:int|const char\*)\s+(vdit_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"vdit_patchify_3d", "vdit_rope_3d", "vdit_attn_full", "vdit_attn_divided_time",
+            "vdit_attn_divided_space", "vdit_status_string", "vdit_device_status", "vdit_version"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_strings(L):
+    assert L.vdit_version() == 10000
+    for s in range(7):
+        assert len(L.vdit_status_string(s)) > 0
+    assert L.vdit_status_string(99) == b"unknown status"
+
+
+def patchify(L, latent=FAKE, tokens=FAKE, dtype=0, N=1, C=4, T=8, H=16, W=16, pt=1, ph=2, pw=2):
+    return L.vdit_patchify_3d(latent, tokens, dtype, N, C, T, H, W, pt, ph, pw, None)
+
+
+def test_patchify_validation(L):
+    assert patchify(L, latent=None) == NULL
+    assert patchify(L, tokens=None) == NULL
+    assert patchify(L, dtype=7) == UNSUP
+    assert patchify(L, N=0) == SHAPE
+    assert patchify(L, pw=-1) == SHAPE
+    assert patchify(L, T=1, pt=2) == SHAPE            # no whole brick along time
+    assert patchify(L, C=100000, pt=4, ph=4, pw=4) == UNSUP   # one brick beyond the staging buffer
+
+
+def rope(L, q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, B=1, Tg=2, Hg=3, Wg=4, heads=2, D=128, split=(44, 42, 42),
+         theta=10000.0):
+    return L.vdit_rope_3d(q, k, qo, ko, B, Tg, Hg, Wg, heads, D, *split, ctypes.c_float(theta), None)
+
+
+def test_rope_validation(L):
+    assert rope(L, q=None) == NULL
+    assert rope(L, ko=None) == NULL
+    # the cheatsheet's rope_3d ValueError: widths must add up to the head width
+    assert rope(L, split=(44, 42, 40)) == SHAPE
+    assert rope(L, split=(43, 43, 42)) == SHAPE
+    assert rope(L, split=(-2, 66, 64)) == SHAPE
+    assert rope(L, Hg=0) == SHAPE
+    assert rope(L, theta=0.0) == SHAPE
+    assert rope(L, D=36, split=(12, 12, 12)) == UNSUP  # not a multiple of 8
+    assert rope(L, q=MIS) == ALIGN
+    assert rope(L, ko=MIS) == ALIGN
+
+
+def attn(L, fn="vdit_attn_full", q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, dims=(1, 256, 2, 128)):
+    f = getattr(L, fn)
+    return f(q, k, v, o, lse, *dims, ctypes.c_float(0.0), None)
+
+
+@pytest.mark.parametrize("fn,dims", [("vdit_attn_full", (1, 256, 2, 128)),
+                                     ("vdit_attn_divided_time", (1, 8, 64, 2, 32)),
+                                     ("vdit_attn_divided_space", (1, 8, 64, 2, 32))])
+def test_attention_validation(L, fn, dims):
+    assert attn(L, fn, dims=dims, q=None) == NULL
+    assert attn(L, fn, dims=dims, o=None) == NULL
+    assert attn(L, fn, dims=dims, v=MIS) == ALIGN
+    assert attn(L, fn, dims=dims, lse=FAKE + 2) == ALIGN
+    bad_d = dims[:-1] + (48,)
+    assert attn(L, fn, dims=bad_d) == UNSUP
+    zero = (0,) + dims[1:]
+    assert attn(L, fn, dims=zero) == SHAPE
+    neg = dims[:1] + (-5,) + dims[2:]
+    assert attn(L, fn, dims=neg) == SHAPE
+
+
+def test_binding_refuses_cpu_tensors(L):
+    """The product path has no CPU fallback: host tensors are refused."""
+    import spacetime_attention_vdit_b200 as v
+    q = torch.zeros((1, 8, 1, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        v.attn_full(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        v.patchify_3d(torch.zeros((1, 1, 1, 2, 2)))
+
+
+def test_build_command_targets_sm100a():
+    from spacetime_attention_vdit_b200 import build
+    cmd = build.command()
+    assert "arch=compute_100a,code=sm_100a" in cmd
+    assert "-lineinfo" in cmd

@@ -118,3 +118,28 @@ def test_generator_blocking_invariant():
     finally:
         synthetic._BLOCK = old
     assert np.array_equal(a, c)
+
+
+def test_divided_rows_match_full_passes():
+    g = np.random.default_rng(12)
+    T, HW = 5, 7
+    q, k, v = (g.standard_normal((2, T * HW, 3, 8)) for _ in range(3))
+    rows = np.array([0, 3, 7, 20, 34])
+    ft, lt = ref.divided_time(q, k, v, T, HW)
+    rt, rl = ref.divided_time_rows(q, k, v, T, HW, rows)
+    assert np.allclose(rt, ft[:, rows], atol=1e-14) and np.allclose(rl, lt[:, :, rows], atol=1e-13)
+    fs, ls = ref.divided_space(q, k, v, T, HW)
+    rs, rsl = ref.divided_space_rows(q, k, v, T, HW, rows)
+    assert np.allclose(rs, fs[:, rows], atol=1e-14) and np.allclose(rsl, ls[:, :, rows], atol=1e-13)
+
+
+def test_rope_token_subset():
+    g = np.random.default_rng(13)
+    grid, split = (3, 4, 5), (12, 10, 10)
+    x = g.standard_normal((2, 60, 2, 32))
+    toks = np.array([0, 5, 19, 33, 59])
+    full = ref.rope_3d(x, grid, split)
+    assert np.array_equal(ref.rope_3d(x[:, toks], grid, split, tokens=toks), full[:, toks])
+    x32 = x.astype(np.float32)
+    assert np.array_equal(ref.rope_3d_fp32(x32[:, toks], grid, split, tokens=toks),
+                          ref.rope_3d_fp32(x32, grid, split)[:, toks])

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 
 from oracle import reference as ref
-import pins
+from tests import pins
 
 # ----------------------------------------------------------------------------
 # the real oracle passes
