@@ -46,6 +46,7 @@ WORKLOADS = {
     # name: (B, T latent frames, H latent, W latent, heads, head_dim, description)
     "480p81_cfg_pair": (2, 21, 60, 104, 40, 128,
                         "81-frame 832x480 clip, CFG pair: 2 x 21x30x52 = 32,760 tokens, 40 heads x 128"),
+    "480p81": (1, 21, 60, 104, 40, 128, "81-frame 832x480 clip: 21x30x52 = 32,760 tokens, 40 heads x 128"),
     "720p81": (1, 21, 90, 160, 40, 128, "81-frame 1280x720 clip: 21x45x80 = 75,600 tokens, 40 heads x 128"),
     "480p17": (1, 5, 60, 104, 12, 128, "17-frame 832x480 clip: 5x30x52 = 7,800 tokens, 12 heads x 128"),
 }
@@ -189,6 +190,27 @@ def oracle_sample(d, budget_s, seed=0):
                       f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy"
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank processes its own clip pair (independent problems, weak scaling)."""
+    return 1000 * rank
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of x over all ranks (the timing rule: the slowest rank sets the time)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -260,7 +282,7 @@ def main():
 
     B, L, Hh, D, Tg, HW = d["B"], d["L"], d["heads"], d["D"], d["Tg"], d["HW"]
     grid = (d["Tg"], d["Hg"], d["Wg"])
-    seed = 1000 * rank  # every rank its own clip pair
+    seed = rank_seed(rank)
     lat_h = torch.from_numpy(synthetic.latent_f32(B, LATENT_C, d["T"], d["H"], d["W"], seed=seed)).pin_memory()
     qb, kb, vb = synthetic.qkv_bf16(B, L, Hh, D, seed=seed)
 
@@ -304,11 +326,7 @@ def main():
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -336,7 +354,7 @@ def main():
 
     full_f, time_f, space_f = step_flops(d)
     flops_step = full_f + time_f + space_f
-    value = world * flops_step * args.steps / (ms * 1e-3) / 1e12
+    value = job_throughput(world, flops_step, args.steps, ms)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -365,7 +383,7 @@ def main():
         t2.record(stream)
         barrier()
         e_ms = max_over_ranks(s2.elapsed_time(t2))
-        e2e = {"value": world * flops_step * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_throughput(world, flops_step, e_steps, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms / e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": e_steps}
 

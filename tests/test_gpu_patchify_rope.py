@@ -70,11 +70,15 @@ def _rope_check(B, grid, heads, D, split, seed=3, tokens=None, scale=1.0):
         x32 = synthetic.bf16_bits_to_f32(bits[:, toks])
         exp32 = synthetic.f32_to_bf16_bits(ref.rope_3d_fp32(x32, grid, split, tokens=toks))
         assert np.array_equal(got, exp32), "not bit-identical to the page-precision rotation"
-        # and within one bf16 ulp of the float64 definition
+        # and within one bf16 ulp of the float64 definition, plus the float32
+        # rounding of the two products (which dominates when they cancel):
+        # |err| <= ulp_bf16(result) + 2^-22 * (|x0| + |x1|)
         exp64 = ref.rope_3d(x32.astype(np.float64), grid, split, tokens=toks)
         gotf = synthetic.bf16_bits_to_f64(got)
-        ulp = np.spacing(np.abs(exp64).astype(np.float32)).astype(np.float64) * 2.0 ** 16
-        assert np.all(np.abs(gotf - exp64) <= ulp + 1e-30)
+        mag = np.maximum(np.abs(exp64), np.abs(gotf)).astype(np.float32)
+        ulp = np.spacing(mag).astype(np.float64) * 2.0 ** 16
+        pair = (np.abs(x32[..., 0::2]) + np.abs(x32[..., 1::2])).astype(np.float64).repeat(2, axis=-1)
+        assert np.all(np.abs(gotf - exp64) <= ulp + 2.0 ** -22 * pair)
     return qd, kd, qo, ko
 
 
