@@ -249,12 +249,13 @@ def run_reference(args, d):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-aux", action="store_true", help="skip the large-batch patchify measurement")
     args = ap.parse_args()
     d = workload_dims(args.workload)
     if args.warmup < 3:
@@ -337,8 +338,9 @@ def main():
     # ---- device-resident timed region
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
     with ClockSampler(local) as clk:
+        time.sleep(0.5)          # nvidia-smi is sampling before the timed region starts
+        barrier()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
@@ -417,6 +419,28 @@ def main():
             r["tflops"] = space_f / (per_row[n] * 1e-3) / 1e12
         rows[n] = r
 
+    # ---- auxiliary: patchify at a size where bandwidth, not launch latency, shows
+    aux = None
+    if not args.no_aux:
+        big = torch.empty((64, LATENT_C, 21, 90, 160), dtype=torch.float32, device=dev).normal_()
+        big_tok = torch.empty((64, 21 * 45 * 80, LATENT_C * 4), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            vd.patchify_3d(big, PATCH, out=big_tok)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        a.record(stream)
+        for _ in range(reps):
+            vd.patchify_3d(big, PATCH, out=big_tok)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        pms = a.elapsed_time(b_) / reps
+        pbytes = 2 * big.numel() * 4
+        aux = {"patchify_64_clips_720p": {"latent": [64, LATENT_C, 21, 90, 160], "ms": pms,
+                                          "gb_s": pbytes / (pms * 1e-3) / 1e9,
+                                          "frac_hbm": pbytes / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                          "bytes": pbytes}}
+        del big, big_tok
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, s, desc = oracle_sample(d, 15.0)
@@ -435,7 +459,7 @@ def main():
                            "l2": "inputs larger than L2: %.2f GB of Q/K/V per step" % (3 * q.numel() * 2 / 1e9),
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "aux": aux,
                 "frac_of_nominal_dense_bf16": achieved / 2250.0}
         print(json.dumps(line), flush=True)
     if world > 1:

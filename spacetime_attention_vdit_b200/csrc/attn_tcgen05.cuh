@@ -9,17 +9,28 @@
 // space pass of divided attention (each frame is a contiguous sequence) and,
 // through a strided tensor map, a time pass with long sequences.
 //
-// One CTA computes one 128-row query tile of one (sequence, head):
-//   warp 0      TMA producer: Q once, then K_j and V_j into an NSTAGE ring;
-//   warp 1      allocates TMEM and issues the UMMAs (one thread):
-//                 S_j = Q K_j^T into one of two TMEM score buffers,
-//                 O  += P_j V_j into the TMEM accumulator;
-//   warps 2..5  softmax, one query row per thread (TMEM lane = row): read S_j,
-//               running max (kept unless it grows by more than 2^8, an exact
-//               rescaling rule), P_j = 2^(s*scale*log2e - m) rounded to bf16
-//               into shared memory, O rescaled in TMEM when the max moved,
-//               and finally O / l to global memory with the row's log-sum-exp.
-// S_{j+1} is computed on the tensor cores while the softmax works on S_j.
+// One CTA computes two 128-row query tiles (256 rows) of one (sequence, head):
+//   warp 0      TMA producer: Q tiles once; K_j into a K ring and V_j into a
+//               V ring (K is needed one P.V product earlier than V);
+//   warp 1      allocates all 512 TMEM columns and issues every UMMA from one
+//               thread: S_i = Q_i K_j^T (smem x smem) into tile i's score
+//               columns, then O_i += P_i V_j with P_i read from TMEM (the
+//               softmax overwrote tile i's scores with bf16 probabilities);
+//   warps 2..5  softmax of query tile 0, warps 6..9 of tile 1, one query row
+//               per thread (TMEM lane = row).
+// The two tiles ping-pong: while one warpgroup exponentiates its scores the
+// tensor core runs the other tile's products.  TMEM columns: S/P of tile i at
+// [128 i, 128 i + 128), O of tile i at [256 + 128 i, ...).
+//
+// Softmax per tile and row: running max m kept unless a new tile raises it by
+// more than 2^8 (exact rescaling rule: P stays below 2^8 and O/l is unchanged);
+// P = 2^(s * scale * log2e - m) rounded to bf16; O rescaled in TMEM only when m
+// moved; at the end O / l and the row's log-sum-exp are written out.
+//
+// Each CTA sweeps the key tiles starting at tile (query block mod tiles), so
+// the CTAs of one head, which run together, read different K/V lines from L2
+// at any moment instead of all hammering the same ones; the online softmax
+// does not depend on the order of the tiles.
 #pragma once
 
 #include <math.h>
@@ -31,6 +42,7 @@ namespace vdit {
 template <int D>
 struct AttnCfg {
   static constexpr int BM = 128;                               // query rows per tile
+  static constexpr int NQ = 2;                                 // query tiles per CTA
   static constexpr int BN = 128;                               // keys per KV tile
   static constexpr int ROWB = (D * 2 >= 128) ? 128 : D * 2;    // bytes per staged row of one D-block
   static constexpr int DBLK = ROWB / 2;                        // elements per D-block
@@ -38,15 +50,16 @@ struct AttnCfg {
   static constexpr uint32_t SWZ = ROWB == 128 ? kSwizzle128 : (ROWB == 64 ? kSwizzle64 : kSwizzle32);
   static constexpr int DB_BYTES = BM * ROWB;                   // one D-block of a 128-row tile
   static constexpr int TILE_BYTES = BM * D * 2;
-  static constexpr int NSTAGE = D >= 128 ? 2 : (D >= 64 ? 3 : 4);
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int NBARS = 1 + 3 * NSTAGE + 2 + 2 + 1 + 1 + 1;
-  static constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 2 * NSTAGE * TILE_BYTES + P_BYTES + NBARS * 8 + 16;
+  static constexpr int NK = D >= 128 ? 3 : 4;                  // K ring stages
+  static constexpr int NV = D >= 128 ? 2 : (D >= 64 ? 3 : 4);  // V ring stages
+  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 3 * NQ + 1;
+  static constexpr int SMEM_BYTES = 1024 + (NQ + NK + NV) * TILE_BYTES + NBARS * 8 + 16;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL = 0;                         // S buffers at columns 0 and 128
-  static constexpr uint32_t O_COL = 256;                       // O accumulator, D columns
+  static constexpr uint32_t S_COL = 0;                         // tile i: scores / P at 128 i
+  static constexpr uint32_t O_COL = 256;                       // tile i: accumulator at 256 + 128 i
   static constexpr uint32_t IDESC_QK = umma_idesc_bf16(BM, BN, 0, 0);  // Q, K both K-major
-  static constexpr uint32_t IDESC_PV = umma_idesc_bf16(BM, D, 0, 1);   // P K-major, V MN-major
+  static constexpr uint32_t IDESC_PV = umma_idesc_bf16(BM, D, 0, 1);   // P (TMEM) K-major, V MN-major
   static_assert(D % 16 == 0 && D >= 32 && D <= 128, "head_dim");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -66,14 +79,14 @@ struct AttnParams {
   int heads;
   int grp;             // see AttnMode
   int mode;
-  int n_qtiles;        // ceil(L / 128)
+  int n_qblocks;       // ceil(L / 256): CTAs per (sequence, head)
   int n_kv;            // ceil(L / 128)
   float scale_log2;    // scale * log2(e)
 };
 
 // Wait sites recorded by the watchdog.
 enum : int {
-  kSiteQFull = 1, kSiteKFull, kSiteVFull, kSiteKvEmpty, kSiteSFull, kSiteSFree, kSitePFull, kSiteODone,
+  kSiteQFull = 1, kSiteKFull, kSiteVFull, kSiteKEmpty, kSiteVEmpty, kSiteSFull, kSitePFull, kSiteODone,
   kSiteDrain
 };
 
@@ -93,54 +106,51 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int si
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
   unsigned char* smem_raw = dyn_smem;
   const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
-  unsigned char* sQ = reinterpret_cast<unsigned char*>(base);
-  unsigned char* sK = sQ + C::TILE_BYTES;
-  unsigned char* sV = sK + C::NSTAGE * C::TILE_BYTES;
-  unsigned char* sP = sV + C::NSTAGE * C::TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  unsigned char* sQ = reinterpret_cast<unsigned char*>(base);      // NQ tiles
+  unsigned char* sK = sQ + C::NQ * C::TILE_BYTES;                  // NK tiles
+  unsigned char* sV = sK + C::NK * C::TILE_BYTES;                  // NV tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::NV * C::TILE_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
-  uint64_t* v_full = k_full + C::NSTAGE;
-  uint64_t* kv_empty = v_full + C::NSTAGE;
-  uint64_t* s_full = kv_empty + C::NSTAGE;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* k_empty = k_full + C::NK;
+  uint64_t* v_full = k_empty + C::NK;
+  uint64_t* v_empty = v_full + C::NV;
+  uint64_t* s_full = v_empty + C::NV;      // [NQ]
+  uint64_t* p_full = s_full + C::NQ;       // [NQ]
+  uint64_t* o_done = p_full + C::NQ;       // [NQ]
+  uint64_t* drain = o_done + C::NQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int tile = blockIdx.x;
-  const int qt = tile % p.n_qtiles;
-  const int bh = tile / p.n_qtiles;
+  const int qb = blockIdx.x % p.n_qblocks;
+  const int bh = blockIdx.x / p.n_qblocks;
   const int h = bh % p.heads;
   const int bb = bh / p.heads;
-  const int q0 = qt * C::BM;
+  const int q0 = qb * (C::NQ * C::BM);
+  const int nq = (q0 + C::BM < p.L) ? 2 : 1;   // query tiles holding rows of the sequence
+  const int n = p.n_kv;
+  const int j0 = qb % n;                       // first key tile of this CTA's sweep
   // tensor-map coordinates of this sequence: (d, head, site, position, batch)
   const int c_site = p.mode == kTime ? bb % p.grp : 0;
   const int c_batch = p.mode == kTime ? bb / p.grp : bb;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < C::NSTAGE; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < C::NK; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < C::NV; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);           // one elected lane per softmax warp
+      mbar_init(&o_done[i], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
-    }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -159,74 +169,121 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+      mbar_arrive_expect_tx(q_full, nq * C::TILE_BYTES);
+      for (int i = 0; i < nq; ++i)
 #pragma unroll
-      for (int db = 0; db < C::NDB; ++db)
-        tma_load_5d(sQ + db * C::DB_BYTES, &tmQ, q_full, db * C::DBLK, h, c_site, q0, c_batch);
-      int issued = 0;
-      for (int j = 0; j < p.n_kv; ++j) {
-        const int st = j % C::NSTAGE;
-        if (j >= C::NSTAGE && !mbar_wait(&kv_empty[st], ((j / C::NSTAGE) - 1) & 1, kSiteKvEmpty)) break;
+        for (int db = 0; db < C::NDB; ++db)
+          tma_load_5d(sQ + i * C::TILE_BYTES + db * C::DB_BYTES, &tmQ, q_full, db * C::DBLK, h, c_site,
+                      q0 + i * C::BM, c_batch);
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int j) -> bool {
+        const int st = j % C::NK;
+        if (j >= C::NK && !mbar_wait(&k_empty[st], ((j / C::NK) - 1) & 1, kSiteKEmpty)) return false;
         mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
 #pragma unroll
         for (int db = 0; db < C::NDB; ++db)
           tma_load_5d(sK + st * C::TILE_BYTES + db * C::DB_BYTES, &tmK, &k_full[st], db * C::DBLK, h, c_site,
-                      j * C::BN, c_batch);
+                      ((j + j0) % n) * C::BN, c_batch);
+        k_issued = j + 1;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j % C::NV;
+        if (j >= C::NV && !mbar_wait(&v_empty[st], ((j / C::NV) - 1) & 1, kSiteVEmpty)) return false;
         mbar_arrive_expect_tx(&v_full[st], C::TILE_BYTES);
 #pragma unroll
         for (int db = 0; db < C::NDB; ++db)
           tma_load_5d(sV + st * C::TILE_BYTES + db * C::DB_BYTES, &tmV, &v_full[st], db * C::DBLK, h, c_site,
-                      j * C::BN, c_batch);
-        issued = j + 1;
+                      ((j + j0) % n) * C::BN, c_batch);
+        v_issued = j + 1;
+        return true;
+      };
+      // K runs one tile ahead of V: K_0, K_1, V_0, K_2, V_1, ...
+      bool ok = load_k(0);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
       // No copy may still be landing in shared memory when the CTA exits.
       mbar_drain(q_full, 0);
-      for (int j = issued - C::NSTAGE < 0 ? 0 : issued - C::NSTAGE; j < issued; ++j) {
-        const int st = j % C::NSTAGE;
-        mbar_drain(&k_full[st], (j / C::NSTAGE) & 1);
-        mbar_drain(&v_full[st], (j / C::NSTAGE) & 1);
-      }
+      for (int j = k_issued - C::NK < 0 ? 0 : k_issued - C::NK; j < k_issued; ++j)
+        mbar_drain(&k_full[j % C::NK], (j / C::NK) & 1);
+      for (int j = v_issued - C::NV < 0 ? 0 : v_issued - C::NV; j < v_issued; ++j)
+        mbar_drain(&v_full[j % C::NV], (j / C::NV) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       constexpr uint32_t SBO = 8 * C::ROWB;       // 8-row core-matrix group stride
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj % C::NSTAGE;
-        if (!mbar_wait(&v_full[st], (jj / C::NSTAGE) & 1, kSiteVFull)) return false;
-        if (!mbar_wait(p_full, jj & 1, kSitePFull)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          // A = P (128 x 16 keys), K-major, 128-byte swizzle, 64 keys per 16 KB block
-          const uint64_t a = umma_sdesc(sPa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
-          // B = V (16 keys x D), MN-major: D-blocks DB_BYTES apart, 8-key groups SBO apart
-          const uint64_t b = umma_sdesc(sVa + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::DB_BYTES, SBO, C::SWZ);
-          umma_ss(tmem + C::O_COL, a, b, C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&kv_empty[st]);
-        umma_commit(o_done);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, kSiteQFull);
-      for (int j = 0; j < p.n_kv && ok; ++j) {
-        const int st = j % C::NSTAGE;
-        const int sb = j & 1;
-        if (!mbar_wait(&k_full[st], (j / C::NSTAGE) & 1, kSiteKFull)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, kSiteSFree)) { ok = false; break; }
-        tc_fence_after();
+      auto qk = [&](int i, int j) {
+        const int st = j % C::NK;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / (C::DBLK / 16)) * C::DB_BYTES + (kk % (C::DBLK / 16)) * 32;
-          const uint64_t a = umma_sdesc(sQa + off, 16, SBO, C::SWZ);
+          const uint64_t a = umma_sdesc(sQa + i * C::TILE_BYTES + off, 16, SBO, C::SWZ);
           const uint64_t b = umma_sdesc(sKa + st * C::TILE_BYTES + off, 16, SBO, C::SWZ);
-          umma_ss(tmem + C::S_COL + sb * C::BN, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + C::S_COL + i * C::BN, a, b, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        umma_commit(&s_full[i]);
+      };
+      auto pv = [&](int i, int j) {
+        const int st = j % C::NV;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          // A = P_i: 16 keys = 8 TMEM columns of packed bf16 pairs
+          // B = V (16 keys x D), MN-major: D-blocks DB_BYTES apart, 8-key groups SBO apart
+          const uint64_t b = umma_sdesc(sVa + st * C::TILE_BYTES + kk * 16 * C::ROWB, C::DB_BYTES, SBO, C::SWZ);
+          umma_ts(tmem + C::O_COL + i * C::BM, tmem + C::S_COL + i * C::BN + kk * 8, b, C::IDESC_PV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&o_done[i]);
+      };
+      bool ok = mbar_wait(q_full, 0, kSiteQFull) && mbar_wait(&k_full[0], 0, kSiteKFull);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < nq; ++i) qk(i, 0);
+        umma_commit(&k_empty[0]);
       }
-      if (ok) issue_pv(p.n_kv - 1);
+      // Event loop: issue whichever product is ready, so that while tile i waits
+      // for its P.V to finish (before its scores may be overwritten) the tensor
+      // core works on the other tile.  npv[i] / nqk[i]: next iteration whose
+      // P.V / QK^T tile i issues; a K or V stage is released once both tiles
+      // have issued the products that read it.
+      int npv[2] = {0, nq > 1 ? 0 : n};
+      int nqk[2] = {1, nq > 1 ? 1 : n};
+      int v_rel = 0, k_rel = 1;
+      unsigned long long t_last = globaltimer_ns();
+      while (ok && (npv[0] < n || npv[1] < n)) {
+        bool progress = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int jp = npv[i];
+          if (jp < n && nqk[i] > jp && mbar_test(&p_full[i], jp & 1) &&
+              mbar_test(&v_full[jp % C::NV], (jp / C::NV) & 1)) {
+            tc_fence_after();
+            pv(i, jp);
+            npv[i] = jp + 1;
+            progress = true;
+            for (const int lo = min(npv[0], npv[1]); v_rel < lo; ++v_rel) umma_commit(&v_empty[v_rel % C::NV]);
+          }
+          const int jq = nqk[i];
+          if (jq < n && npv[i] >= jq && mbar_test(&o_done[i], (jq - 1) & 1) &&
+              mbar_test(&k_full[jq % C::NK], (jq / C::NK) & 1)) {
+            tc_fence_after();
+            qk(i, jq);
+            nqk[i] = jq + 1;
+            progress = true;
+            for (const int lo = min(nqk[0], nqk[1]); k_rel < lo; ++k_rel) umma_commit(&k_empty[k_rel % C::NK]);
+          }
+        }
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else if (watchdog_tripped() || globaltimer_ns() - t_last > kWaitLimitNs) {
+          watchdog_trip(kSiteODone);
+          ok = false;
+        }
+      }
       // every UMMA issued above has finished before TMEM is released
       umma_commit(drain);
       mbar_drain(drain, 0);
@@ -234,24 +291,24 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- softmax
+    const int tile = (warp - 2) >> 2;             // warps 2..5 -> tile 0, 6..9 -> tile 1
     const int quad = warp & 3;                    // TMEM lanes this warp may touch
     const int row = quad * 32 + lane;             // query row within the tile
-    const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t t_s = tl + C::S_COL + tile * C::BN;
+    const uint32_t t_o = tl + C::O_COL + tile * C::BM;
     float m_use = -INFINITY;                      // max used for the exponentials (log2 units)
     float l_sum = 0.f;
-    bool ok = true;
-    for (int j = 0; j < p.n_kv; ++j) {
-      const int sb = j & 1;
-      if (!warp_wait(&s_full[sb], (j >> 1) & 1, kSiteSFull)) { ok = false; break; }
+    bool ok = tile < nq;
+    for (int j = 0; j < n && ok; ++j) {
+      if (!warp_wait(&s_full[tile], j & 1, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tlane + C::S_COL + sb * C::BN + c * 32, s[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, s[c]);
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
 
-      const int valid = p.L - j * C::BN;          // keys of this tile inside the sequence
+      const int valid = p.L - ((j + j0) % n) * C::BN;   // keys of this tile inside the sequence
       if (valid < C::BN) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -259,11 +316,15 @@ __global__ void __launch_bounds__(192, 1)
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      float mp[8];                                // eight independent max chains
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+        for (int e = 0; e < 32; ++e) mp[e & 7] = fmaxf(mp[e & 7], __uint_as_float(s[c][e]));
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_new = mx * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -274,52 +335,47 @@ __global__ void __launch_bounds__(192, 1)
         m_use = m_new;
         rescale = true;
       }
-      const float neg_m = -m_use;
-      float rsum = 0.f;
-      uint32_t pk[64];                            // P row as bf16 pairs
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};   // four independent packed sum chains
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][e]), p.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][e + 1]), p.scale_log2, neg_m));
-          rsum += p0 + p1;
-          pk[(c * 32 + e) >> 1] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), sc2, nm2);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          sp[(e >> 1) & 3] = fadd2(sp[(e >> 1) & 3], pr);
+          pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
         }
-
-      // P and O may be touched only once the previous P.V product is done.
-      if (j >= 1 && !warp_wait(o_done, (j - 1) & 1, kSiteODone)) { ok = false; break; }
-      tc_fence_after();
-      // P row -> shared memory, K-major, 128-byte swizzle: key block kb (64 keys,
-      // 16 KB), 16-byte chunk c of the row stored at chunk c ^ (row % 8).
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int kb = ch >> 3, c = ch & 7;
-        uint4* dst = reinterpret_cast<uint4*>(sP + kb * 16384 + row * 128 + ((c ^ (row & 7)) << 4));
-        *dst = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+        // P over this tile's own score columns: keys 32c .. 32c+31 -> 16 columns
+        tmem_st16(t_s + c * 16, pk);
       }
+      const float2 s01 = fadd2(fadd2(sp[0], sp[1]), fadd2(sp[2], sp[3]));
+      const float rsum = s01.x + s01.y;
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tlane + C::O_COL + c * 32, o);
+          tmem_ld32(t_o + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tlane + C::O_COL + c * 32, o);
+          tmem_st32(t_o + c * 32, o);
         }
-        tmem_st_wait();
       }
       l_sum = l_sum * alpha + rsum;
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[tile]);
     }
 
     // ------------------------------------------------------------- epilogue
-    if (ok && warp_wait(o_done, (p.n_kv - 1) & 1, kSiteODone)) {
+    if (ok && warp_wait(&o_done[tile], (n - 1) & 1, kSiteODone)) {
       tc_fence_after();
-      const int i = q0 + row;                     // position in the sequence
+      const int i = q0 + tile * C::BM + row;      // position in the sequence
       const float inv_l = 1.f / l_sum;
       long long token;
       if (p.mode == kTime) {
@@ -332,7 +388,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tlane + C::O_COL + c * 32, o);
+        tmem_ld32(t_o + c * 32, o);
         tmem_ld_wait();
         if (i < p.L) {
 #pragma unroll

@@ -6,17 +6,18 @@
 // site s, head h) the tokens {t*HW + s : t < T}.  With T = 21 latent frames each
 // such problem is tiny (21 x 21 scores) and there are B*HW*heads of them, so
 // the pass moves Q, K, V and O once through HBM at an arithmetic intensity of
-// about 10 flop/byte: it is bandwidth-bound, not tensor-bound.
+// about 10 flop/byte: it is bandwidth-bound, and is built to keep HBM busy.
 //
-// Design: one warp owns one (b, s, h) problem at a time.  It copies the T rows of
-// Q, K and V (each row is one head's 256 contiguous bytes; rows are HW*heads*D
-// elements apart) into its own swizzled shared-memory slots with 16-byte
-// cp.async, computes S = Q K^T and O = P V with warp-level bf16 tensor-core
-// MMAs (m16n8k16, fp32 accumulation) on rows padded to TP, keeps the softmax in
-// registers, stages O back through shared memory and writes it with 16-byte
-// stores.  Eight warps per CTA (fewer when T > 32) keep the other problems'
-// loads in flight while one computes; consecutive warps take consecutive heads of the same site, so a CTA
-// streams contiguous runs of each token row.  Pad rows of K and V are zero.
+// Design: a producer warp streams problems into a ring of shared-memory stages
+// with TMA - one 5-D box per D-block per tensor: {D-block, 1 head, 1 site, TP
+// frames, 1 batch} over the view {D, heads, sites, frames, batch}, so the box
+// gathers the site's T rows (HW*heads*D elements apart) in one copy and rows
+// TP > T arrive as zeros.  Each consumer warp owns two stages and alternates
+// between them, so its next problem is in flight while it computes the current
+// one.  A consumer computes S = Q K^T and O = P V with warp-level bf16
+// tensor-core MMAs (m16n8k16, fp32 accumulation) on rows padded to TP, keeps the
+// softmax in registers, stages O over the stage's Q rows and writes it with
+// 16-byte stores, then releases the stage to the producer.
 #pragma once
 
 #include "ptx.cuh"
@@ -25,30 +26,31 @@ namespace vdit {
 
 template <int D, int TP>
 struct TimeCfg {
-  static constexpr int CPR = D / 8;                          // 16-byte chunks per row
-  static constexpr int ROW_BYTES = D * 2;
-  static constexpr int SLOT_BYTES = TP * ROW_BYTES;          // one tensor's rows
-  static constexpr int WARP_BYTES = 3 * SLOT_BYTES;          // Q, K, V
-  // eight warps when their slots fit in 200 KB, fewer for long padded rows
-  static constexpr int WARPS = (200 * 1024) / WARP_BYTES >= 8 ? 8 : (200 * 1024) / WARP_BYTES;
-  static constexpr int SMEM_BYTES = WARPS * WARP_BYTES;
+  static constexpr int ROWB = (D * 2 >= 128) ? 128 : D * 2;   // bytes per row of one D-block
+  static constexpr int DBLK = ROWB / 2;                       // elements per D-block
+  static constexpr int NDB = D / DBLK;                        // D-blocks
+  static constexpr int CPB = ROWB / 16;                       // 16-byte chunks per D-block row
+  static constexpr int REGION = TP * ROWB;                    // one D-block of one tensor
+  static constexpr int TENSOR_BYTES = NDB * REGION;           // = TP * D * 2
+  static constexpr int STAGE_BYTES = 3 * TENSOR_BYTES;        // Q, K, V
+  static constexpr int NSTAGE_MAX = (196608 / STAGE_BYTES) & ~1;
+  static constexpr int NSTAGE = NSTAGE_MAX > 16 ? 16 : NSTAGE_MAX;
+  static constexpr int NC = NSTAGE / 2;                       // consumer warps, two stages each
+  static constexpr int THREADS = 32 * (1 + NC);
+  static constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8;
   static_assert(D % 16 == 0 && D >= 32 && D <= 128, "head_dim");
   static_assert(TP == 16 || TP == 32 || TP == 64, "padded length");
+  static_assert(NSTAGE >= 2, "stages");
 };
 
-// Physical 16-byte chunk of logical chunk c in row r: XOR-swizzled so that the
-// eight rows an ldmatrix reads at one column fall in different banks.
-template <int D>
-__device__ __forceinline__ int time_swz(int r, int c) {
-  if constexpr (D / 8 >= 8) return c ^ (r & 7);
-  else return c ^ ((r >> 1) & 3);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+// Byte offset of 16-byte chunk c (0 .. D/8-1) of row r inside one tensor of a
+// stage, as the TMA box lays it out: D-block c / CPB, rows of ROWB bytes, the
+// chunk index XOR-swizzled with the row (128-byte or 64-byte swizzle).
+template <int D, int TP>
+__device__ __forceinline__ uint32_t time_off(int r, int c) {
+  using C = TimeCfg<D, TP>;
+  const int key = C::ROWB == 128 ? (r & 7) : ((r >> 1) & 3);
+  return (uint32_t)((c / C::CPB) * C::REGION + r * C::ROWB + (((c % C::CPB) ^ key) << 4));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -71,9 +73,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 }
 
 struct TimeParams {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k;
-  const __nv_bfloat16* v;
   __nv_bfloat16* o;
   float* lse;           // may be null; [B, heads, T*HW]
   int B, T, HW, heads;
@@ -81,49 +80,86 @@ struct TimeParams {
 };
 
 template <int D, int TP>
-__global__ void __launch_bounds__(256) attn_time_short_kernel(const TimeParams p) {
+__global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
+    attn_time_short_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const TimeParams p) {
   using C = TimeCfg<D, TP>;
-  unsigned char* smem_raw = dyn_smem;
-  if (watchdog_tripped()) return;
+  const uintptr_t base = (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023);
+  unsigned char* stages = reinterpret_cast<unsigned char*>(base);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + C::NSTAGE * C::STAGE_BYTES);
+  uint64_t* empty = full + C::NSTAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* wbase = smem_raw + warp * C::WARP_BYTES;
-  unsigned char* sQ = wbase;
-  unsigned char* sK = wbase + C::SLOT_BYTES;
-  unsigned char* sV = wbase + 2 * C::SLOT_BYTES;
-  const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
 
-  // zero the whole slot once: rows >= T stay zero for every problem
-  for (int i = lane; i < C::WARP_BYTES / 16; i += 32)
-    reinterpret_cast<uint4*>(wbase)[i] = make_uint4(0, 0, 0, 0);
-  __syncwarp();
-
-  const int T = p.T;
   const long long n_units = (long long)p.B * p.HW * p.heads;
+  // this CTA's contiguous run of problems
+  const long long u_begin = n_units * blockIdx.x / gridDim.x;
+  const long long u_end = n_units * (blockIdx.x + 1) / gridDim.x;
+  const int n_local = (int)(u_end - u_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // problem k of this CTA -> stage (k % NC) * 2 + (k / NC) % 2, consumer k % NC
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int issued = 0;
+      for (int k = 0; k < n_local; ++k) {
+        const int st = (k % C::NC) * 2 + ((k / C::NC) & 1);
+        const int use = k / (2 * C::NC);                    // earlier fills of this stage
+        if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, 20)) break;
+        const long long u = u_begin + k;
+        const int h = (int)(u % p.heads);
+        const long long bs = u / p.heads;
+        const int s = (int)(bs % p.HW);
+        const int b = (int)(bs / p.HW);
+        unsigned char* sb = stages + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+#pragma unroll
+        for (int db = 0; db < C::NDB; ++db) {
+          tma_load_5d(sb + 0 * C::TENSOR_BYTES + db * C::REGION, &tmQ, &full[st], db * C::DBLK, h, s, 0, b);
+          tma_load_5d(sb + 1 * C::TENSOR_BYTES + db * C::REGION, &tmK, &full[st], db * C::DBLK, h, s, 0, b);
+          tma_load_5d(sb + 2 * C::TENSOR_BYTES + db * C::REGION, &tmV, &full[st], db * C::DBLK, h, s, 0, b);
+        }
+        issued = k + 1;
+      }
+      // drain: the last fill of every stage has landed before the CTA exits
+      for (int k = issued - 2 * C::NC < 0 ? 0 : issued - 2 * C::NC; k < issued; ++k) {
+        const int st = (k % C::NC) * 2 + ((k / C::NC) & 1);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[st], (k / (2 * C::NC)) & 1))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) { watchdog_trip(21); break; }
+      }
+    }
+    return;
+  }
+
+  const int cw = warp - 1;                   // consumer index
+  const int T = p.T;
   const long long row_stride = (long long)p.HW * p.heads * D;    // elements between frames
   const int n_mt = (T + 15) / 16;
-
-  for (long long u = (long long)blockIdx.x * C::WARPS + warp; u < n_units;
-       u += (long long)gridDim.x * C::WARPS) {
+  const int g8 = lane >> 2;                  // fragment row within an 8-row group
+  const int q2 = (lane & 3) * 2;             // fragment column pair
+  int j = 0;                                 // this consumer's problem count
+  for (int k = cw; k < n_local; k += C::NC, ++j) {
+    const int st = cw * 2 + (j & 1);
+    if (!mbar_wait(&full[st], (j >> 1) & 1, 22)) break;
+    unsigned char* sb = stages + st * C::STAGE_BYTES;
+    const uint32_t aQ = smem_u32(sb), aK = aQ + C::TENSOR_BYTES, aV = aQ + 2 * C::TENSOR_BYTES;
+    const long long u = u_begin + k;
     const int h = (int)(u % p.heads);
     const long long bs = u / p.heads;
     const int s = (int)(bs % p.HW);
     const int b = (int)(bs / p.HW);
-    const long long first = (((long long)b * T * p.HW + s) * p.heads + h) * D;  // element of (t = 0)
 
-    // ---- load T rows of Q, K, V
-    for (int i = lane; i < T * C::CPR; i += 32) {
-      const int t = i / C::CPR, c = i - t * C::CPR;
-      const long long g = first + t * row_stride + c * 8;
-      const uint32_t so = t * C::ROW_BYTES + (time_swz<D>(t, c) << 4);
-      cp_async16(aQ + so, p.q + g);
-      cp_async16(aK + so, p.k + g);
-      cp_async16(aV + so, p.v + g);
-    }
-    cp_async_wait_all();
-    __syncwarp();
-
-    const int g8 = lane >> 2;           // fragment row within an 8-row group
-    const int q2 = (lane & 3) * 2;      // fragment column pair
     for (int mt = 0; mt < n_mt; ++mt) {
       // ---- S = Q K^T for rows mt*16 .. mt*16+15, all TP key columns
       float sacc[TP / 8][4];
@@ -132,15 +168,12 @@ __global__ void __launch_bounds__(256) attn_time_short_kernel(const TimeParams p
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t a0, a1, a2, a3;
-        {
-          const int r = mt * 16 + (lane & 15), c = kk * 2 + (lane >> 4);
-          ldsm_x4(aQ + r * C::ROW_BYTES + (time_swz<D>(r, c) << 4), a0, a1, a2, a3);
-        }
+        ldsm_x4(aQ + time_off<D, TP>(mt * 16 + (lane & 15), kk * 2 + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
         for (int np = 0; np < TP / 16; ++np) {
           uint32_t b0, b1, b2, b3;
-          const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3), c = kk * 2 + ((lane >> 3) & 1);
-          ldsm_x4(aK + r * C::ROW_BYTES + (time_swz<D>(r, c) << 4), b0, b1, b2, b3);
+          ldsm_x4(aK + time_off<D, TP>(np * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)),
+                  b0, b1, b2, b3);
           mma_bf16_16816(sacc[2 * np], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(sacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
         }
@@ -190,24 +223,23 @@ __global__ void __launch_bounds__(256) attn_time_short_kernel(const TimeParams p
 #pragma unroll
         for (int dp = 0; dp < D / 16; ++dp) {
           uint32_t b0, b1, b2, b3;
-          const int r = k2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), c = dp * 2 + (lane >> 4);
-          ldsm_x4_t(aV + r * C::ROW_BYTES + (time_swz<D>(r, c) << 4), b0, b1, b2, b3);
+          ldsm_x4_t(aV + time_off<D, TP>(k2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), dp * 2 + (lane >> 4)),
+                    b0, b1, b2, b3);
           mma_bf16_16816(oacc[2 * dp], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(oacc[2 * dp + 1], a0, a1, a2, a3, b2, b3);
         }
       }
-      // ---- normalise, stage rows < T of this m-tile over their (consumed) Q rows
+      // ---- normalise; stage rows < T of this m-tile over their (consumed) Q rows
       __syncwarp();
       const float inv0 = 1.f / l0, inv1 = 1.f / l1;
       const int r0 = mt * 16 + g8, r1 = r0 + 8;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int c = n;                        // 8 columns = one 16-byte chunk
+      for (int n = 0; n < D / 8; ++n) {       // 8 columns = one 16-byte chunk
         if (r0 < T)
-          *reinterpret_cast<uint32_t*>(sQ + r0 * C::ROW_BYTES + (time_swz<D>(r0, c) << 4) + q2 * 2) =
+          *reinterpret_cast<uint32_t*>(sb + time_off<D, TP>(r0, n) + q2 * 2) =
               pack_bf16x2(oacc[n][0] * inv0, oacc[n][1] * inv0);
         if (r1 < T)
-          *reinterpret_cast<uint32_t*>(sQ + r1 * C::ROW_BYTES + (time_swz<D>(r1, c) << 4) + q2 * 2) =
+          *reinterpret_cast<uint32_t*>(sb + time_off<D, TP>(r1, n) + q2 * 2) =
               pack_bf16x2(oacc[n][2] * inv1, oacc[n][3] * inv1);
       }
       if (p.lse != nullptr && (lane & 3) == 0) {
@@ -218,13 +250,17 @@ __global__ void __launch_bounds__(256) attn_time_short_kernel(const TimeParams p
       __syncwarp();
     }
 
-    // ---- write O rows back to their tokens
-    for (int i = lane; i < T * C::CPR; i += 32) {
-      const int t = i / C::CPR, c = i - t * C::CPR;
-      const uint4 val = *reinterpret_cast<const uint4*>(sQ + t * C::ROW_BYTES + (time_swz<D>(t, c) << 4));
+    // ---- write O rows back to their tokens, then hand the stage back
+    const long long first = (((long long)b * T * p.HW + s) * p.heads + h) * D;   // element of t = 0
+    for (int i = lane; i < T * (D / 8); i += 32) {
+      const int t = i / (D / 8), c = i - t * (D / 8);
+      const uint4 val = *reinterpret_cast<const uint4*>(sb + time_off<D, TP>(t, c));
       *reinterpret_cast<uint4*>(p.o + first + t * row_stride + c * 8) = val;
     }
+    // the stage's next fill is an async-proxy write over these generic-proxy accesses
+    fence_proxy_async_smem();
     __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
   }
 }
 

@@ -18,9 +18,10 @@ namespace vdit {
 // One CTA owns a run of WC bricks that share (n, t', h') - consecutive tokens,
 // so its output is one contiguous span of WC*F elements (F = C*pt*ph*pw).  The
 // CTA first copies the C*pt*ph latent rows those bricks cover (each a
-// contiguous run of WC*pw elements along W) into shared memory with coalesced
-// loads, then writes the output span in order with coalesced stores, reading
-// each element's source from shared memory by the brick index formula.
+// contiguous run of WC*pw elements along W) into shared memory, one warp per
+// row with the lanes sweeping the row; then each warp writes whole bricks, the
+// lanes sweeping the brick's F features in order, each feature's source found
+// in a per-CTA table of staged offsets.  No division runs per element.
 
 struct PatchifyShape {
   int N, C, T, H, W, pt, ph, pw;
@@ -30,16 +31,24 @@ struct PatchifyShape {
   int n_wchunks;    // ceil(Wg / WC)
 };
 
+constexpr int kPatchifyThreads = 256;
+
 template <typename E>
-__global__ void __launch_bounds__(256) patchify3d_kernel(const E* __restrict__ latent, E* __restrict__ tokens,
-                                                         PatchifyShape s) {
-  E* rows = reinterpret_cast<E*>(dyn_smem);
+__global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* __restrict__ latent,
+                                                                      E* __restrict__ tokens, PatchifyShape s) {
+  // dynamic shared memory: F staged-row offsets (int), then the staged rows
+  int* src_off = reinterpret_cast<int*>(dyn_smem);
+  E* rows = reinterpret_cast<E*>(dyn_smem + ((s.F * sizeof(int) + 15) & ~size_t(15)));
   if (watchdog_tripped()) return;
 
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int rowlen = s.WC * s.pw;                 // elements per staged row
   const int nrows = s.C * s.pt * s.ph;
+  // feature f = ((c*pt + dt)*ph + dh)*pw + dw  reads staged row (c*pt + dt)*ph + dh at dw
+  for (int f = threadIdx.x; f < s.F; f += blockDim.x) src_off[f] = (f / s.pw) * rowlen + f % s.pw;
 
-  for (long long job = blockIdx.x; job < (long long)s.N * s.Tg * s.Hg * s.n_wchunks; job += gridDim.x) {
+  const long long n_jobs = (long long)s.N * s.Tg * s.Hg * s.n_wchunks;
+  for (long long job = blockIdx.x; job < n_jobs; job += gridDim.x) {
     const int wc = (int)(job % s.n_wchunks);
     long long r = job / s.n_wchunks;
     const int hq = (int)(r % s.Hg);
@@ -50,32 +59,27 @@ __global__ void __launch_bounds__(256) patchify3d_kernel(const E* __restrict__ l
     const int nb = min(s.WC, s.Wg - w0);          // bricks in this chunk
     const int len = nb * s.pw;                    // valid elements per staged row
 
-    // stage latent rows (c, dt, dh) -> rows[((c*pt + dt)*ph + dh) * rowlen + x]
-    for (int i = threadIdx.x; i < nrows * len; i += blockDim.x) {
-      const int row = i / len, x = i - row * len;
+    __syncthreads();                              // previous job's rows consumed; table written
+    // stage latent rows (c, dt, dh): one warp per row
+    for (int row = warp; row < nrows; row += nwarps) {
       const int dh = row % s.ph;
-      const int dt = (row / s.ph) % s.pt;
-      const int c = row / (s.ph * s.pt);
-      const long long src =
-          ((((long long)n * s.C + c) * s.T + (tq * s.pt + dt)) * s.H + (hq * s.ph + dh)) * s.W + (long long)w0 * s.pw + x;
-      rows[row * rowlen + x] = latent[src];
+      const int cdt = row / s.ph;
+      const int dt = cdt % s.pt;
+      const int c = cdt / s.pt;
+      const E* src = latent + ((((long long)n * s.C + c) * s.T + (tq * s.pt + dt)) * s.H + (hq * s.ph + dh)) *
+                                  (long long)s.W + (long long)w0 * s.pw;
+      E* dst = rows + row * rowlen;
+      for (int x = lane; x < len; x += 32) dst[x] = src[x];
     }
     __syncthreads();
 
-    // write the contiguous output span of nb tokens
-    const long long tok0 = ((long long)n * s.Tg + tq) * s.Hg * s.Wg + (long long)hq * s.Wg + w0;
-    E* out = tokens + tok0 * s.F;
-    const int ppw = s.ph * s.pw, pppw = s.pt * ppw;
-    for (int i = threadIdx.x; i < nb * s.F; i += blockDim.x) {
-      const int b = i / s.F, f = i - b * s.F;
-      const int c = f / pppw;
-      const int rem = f - c * pppw;
-      const int dt = rem / ppw;
-      const int dh = (rem / s.pw) % s.ph;
-      const int dw = rem % s.pw;
-      out[i] = rows[((c * s.pt + dt) * s.ph + dh) * rowlen + b * s.pw + dw];
+    // write the contiguous output span of nb tokens: one warp per brick
+    E* out = tokens + (((long long)n * s.Tg + tq) * s.Hg * s.Wg + (long long)hq * s.Wg + w0) * s.F;
+    for (int b = warp; b < nb; b += nwarps) {
+      const E* from = rows + b * s.pw;
+      E* to = out + (long long)b * s.F;
+      for (int f = lane; f < s.F; f += 32) to[f] = from[src_off[f]];
     }
-    __syncthreads();
   }
 }
 

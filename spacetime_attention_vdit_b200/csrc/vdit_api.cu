@@ -68,10 +68,11 @@ EncodeTiledFn encode_tiled() {
 }
 
 // 5-D view {head_dim, heads, sites, positions, batches} of a bf16 [.., heads, D]
-// token array; box {DBLK, 1, 1, 128, 1}.  Rows outside the positions extent
+// token array; box {DBLK, 1, 1, box_rows, 1}.  Rows outside the positions extent
 // read as zero.
 bool make_qkv_map(CUtensorMap* map, const void* base, int D, int heads, long long sites, long long positions,
-                  long long batches, long long site_stride_el, long long pos_stride_el, long long batch_stride_el) {
+                  long long batches, long long site_stride_el, long long pos_stride_el, long long batch_stride_el,
+                  int box_rows = 128) {
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return false;
   const int rowb = D * 2 >= 128 ? 128 : D * 2;
@@ -79,7 +80,7 @@ bool make_qkv_map(CUtensorMap* map, const void* base, int D, int heads, long lon
                               (cuuint64_t)batches};
   const cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)site_stride_el * 2, (cuuint64_t)pos_stride_el * 2,
                                  (cuuint64_t)batch_stride_el * 2};
-  const cuuint32_t box[5] = {(cuuint32_t)(rowb / 2), 1, 1, 128, 1};
+  const cuuint32_t box[5] = {(cuuint32_t)(rowb / 2), 1, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle sw = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -134,12 +135,12 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
   p.heads = heads;
   p.grp = grp;
   p.mode = mode;
-  p.n_qtiles = (L + C::BM - 1) / C::BM;
+  p.n_qblocks = (L + C::NQ * C::BM - 1) / (C::NQ * C::BM);
   p.n_kv = (L + C::BN - 1) / C::BN;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const long long grid = (long long)n_seq * heads * p.n_qtiles;
+  const long long grid = (long long)n_seq * heads * p.n_qblocks;
   if (grid > 0x7fffffffLL) return VDIT_ERR_SHAPE;
-  attn_fwd_tcgen05_kernel<D><<<(unsigned)grid, 192, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  attn_fwd_tcgen05_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return last_launch_status();
 }
 
@@ -154,7 +155,7 @@ int dispatch_tcgen05(int D, const void* q, const void* k, const void* v, void* o
 }
 
 template <int D, int TP>
-int launch_time_short(const TimeParams& p, cudaStream_t stream) {
+int launch_time_short(const void* q, const void* k, const void* v, const TimeParams& p, cudaStream_t stream) {
   using C = TimeCfg<D, TP>;
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -162,19 +163,27 @@ int launch_time_short(const TimeParams& p, cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(mu);
     if (!ensure_smem(attn_time_short_kernel<D, TP>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
   }
+  // view {D, heads, sites, frames, batch}; one box = one site's TP frames of one head
+  const long long tok = (long long)p.heads * D;
+  CUtensorMap mq, mk, mv;
+  const long long site_st = tok, frame_st = tok * p.HW, batch_st = tok * p.HW * p.T;
+  if (!make_qkv_map(&mq, q, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP) ||
+      !make_qkv_map(&mk, k, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP) ||
+      !make_qkv_map(&mv, v, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP))
+    return VDIT_ERR_CUDA;
   const long long units = (long long)p.B * p.HW * p.heads;
-  const long long want = (units + C::WARPS - 1) / C::WARPS;
-  const long long cap = (long long)sm_count() * 8;   // grid-stride beyond this
-  const unsigned grid = (unsigned)(want < cap ? want : cap);
-  attn_time_short_kernel<D, TP><<<grid, C::WARPS * 32, C::SMEM_BYTES, stream>>>(p);
+  const long long cap = (long long)sm_count();       // one persistent CTA per SM
+  const unsigned grid = (unsigned)(units < cap ? units : cap);
+  attn_time_short_kernel<D, TP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return last_launch_status();
 }
 
 template <int D>
-int dispatch_time_short_tp(const TimeParams& p, cudaStream_t stream) {
-  if (p.T <= 16) return launch_time_short<D, 16>(p, stream);
-  if (p.T <= 32) return launch_time_short<D, 32>(p, stream);
-  return launch_time_short<D, 64>(p, stream);
+int dispatch_time_short_tp(const void* q, const void* k, const void* v, const TimeParams& p,
+                           cudaStream_t stream) {
+  if (p.T <= 16) return launch_time_short<D, 16>(q, k, v, p, stream);
+  if (p.T <= 32) return launch_time_short<D, 32>(q, k, v, p, stream);
+  return launch_time_short<D, 64>(q, k, v, p, stream);
 }
 
 float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)D); }
@@ -243,16 +252,26 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, 
   s.F = (int)F;
   s.WC = (int)std::min<long long>(s.Wg, kStage / brick_bytes);
   s.n_wchunks = (s.Wg + s.WC - 1) / s.WC;
-  const int smem = (int)((long long)C * pt * ph * s.WC * pw * esz);
+  const int smem = (int)(((F * 4 + 15) & ~15LL) + (long long)C * pt * ph * s.WC * pw * esz);
   const long long jobs = (long long)N * s.Tg * s.Hg * s.n_wchunks;
   const long long cap = (long long)sm_count() * 16;
   const unsigned grid = (unsigned)(jobs < cap ? jobs : cap);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  {
+    // staged rows (<= 32 KB) plus the feature offset table (<= 32 KB)
+    static bool done_f[kMaxDevices] = {}, done_b[kMaxDevices] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ensure_smem(patchify3d_kernel<float>, 2 * kStage + 16, done_f) ||
+        !ensure_smem(patchify3d_kernel<__nv_bfloat16>, 2 * kStage + 16, done_b))
+      return VDIT_ERR_CUDA;
+  }
   if (dtype == VDIT_F32)
-    patchify3d_kernel<float><<<grid, 256, smem, st>>>(static_cast<const float*>(latent), static_cast<float*>(tokens), s);
+    patchify3d_kernel<float><<<grid, kPatchifyThreads, smem, st>>>(static_cast<const float*>(latent),
+                                                                   static_cast<float*>(tokens), s);
   else
-    patchify3d_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(latent),
-                                                              static_cast<__nv_bfloat16*>(tokens), s);
+    patchify3d_kernel<__nv_bfloat16><<<grid, kPatchifyThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(latent), static_cast<__nv_bfloat16*>(tokens), s);
   return last_launch_status();
 }
 
@@ -310,17 +329,14 @@ int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o,
   if (T > 64)  // long clips: the tensor-core kernel over a strided view, one sequence per site
     return dispatch_tcgen05(head_dim, q, k, v, o, lse, kTime, B * HW, T, HW, heads, sc, st);
   TimeParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = B; p.T = T; p.HW = HW; p.heads = heads;
   p.scale_log2 = sc * 1.4426950408889634f;
   switch (head_dim) {
-    case 32: return dispatch_time_short_tp<32>(p, st);
-    case 64: return dispatch_time_short_tp<64>(p, st);
-    case 128: return dispatch_time_short_tp<128>(p, st);
+    case 32: return dispatch_time_short_tp<32>(q, k, v, p, st);
+    case 64: return dispatch_time_short_tp<64>(q, k, v, p, st);
+    case 128: return dispatch_time_short_tp<128>(q, k, v, p, st);
     default: return VDIT_ERR_UNSUPPORTED;
   }
 }

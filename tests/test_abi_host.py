@@ -113,3 +113,43 @@ def test_build_command_targets_sm100a():
     cmd = build.command()
     assert "arch=compute_100a,code=sm_100a" in cmd
     assert "-lineinfo" in cmd
+
+
+def test_register_budget_fits_each_sm_subpartition():
+    """Every kernel's registers x the warps one SM sub-partition receives fit its
+    16,384 registers (warps of a CTA are spread round-robin over 4 sub-partitions),
+    so no launch can fail for lack of registers.  Uses ptxas's own report."""
+    import shutil
+    import subprocess
+    from spacetime_attention_vdit_b200 import build
+    if shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"):
+        pytest.skip("nvcc not available")
+    out = "/tmp/vdit_regcheck.so"
+    res = subprocess.run(build.command(ptxas_verbose=True, out=out), capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr[-2000:]
+    regs = {}
+    name = None
+    for line in res.stderr.splitlines():
+        m = re.search(r"Compiling entry function '(\w+)'", line)
+        if m:
+            name = m.group(1)
+        m = re.search(r"Used (\d+) registers", line)
+        if m and name:
+            regs[name] = int(m.group(1))
+    threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256}
+
+    def block_of(kname):
+        for key, t in threads.items():
+            if key in kname:
+                return t
+        m = re.search(r"attn_time_short_kernelILi(\d+)ELi(\d+)", kname)
+        D, TP = int(m.group(1)), int(m.group(2))
+        stage = 3 * TP * D * 2
+        nstage = min(16, (196608 // stage) & ~1)
+        return 32 * (1 + nstage // 2)
+    assert regs, "no ptxas report"
+    for kname, r in regs.items():
+        warps = block_of(kname) // 32
+        per_sub = -(-warps // 4)                  # warps on the fullest sub-partition
+        alloc = -(-r // 8) * 8                    # registers are granted in multiples of 8
+        assert per_sub * 32 * alloc <= 16384, (kname, r, block_of(kname))
