@@ -12,9 +12,10 @@
 // with TMA - one 5-D box per D-block per tensor: {D-block, 1 head, 1 site, TP
 // frames, 1 batch} over the view {D, heads, sites, frames, batch}, so the box
 // gathers the site's T rows (HW*heads*D elements apart) in one copy and rows
-// TP > T arrive as zeros.  Each consumer warp owns two stages and alternates
-// between them, so its next problem is in flight while it computes the current
-// one.  A consumer computes S = Q K^T and O = P V with warp-level bf16
+// TP > T arrive as zeros.  Each consumer group (two warps when T > 16, one per
+// 16-row m-tile; one warp otherwise) owns two stages and alternates between
+// them, so its next problem is in flight while it computes the current one.
+// A consumer warp computes S = Q K^T and O = P V with warp-level bf16
 // tensor-core MMAs (m16n8k16, fp32 accumulation) on rows padded to TP, keeps the
 // softmax in registers, stages O over the stage's Q rows and writes it with
 // 16-byte stores, then releases the stage to the producer.
@@ -35,7 +36,9 @@ struct TimeCfg {
   static constexpr int STAGE_BYTES = 3 * TENSOR_BYTES;        // Q, K, V
   static constexpr int NSTAGE_MAX = (196608 / STAGE_BYTES) & ~1;
   static constexpr int NSTAGE = NSTAGE_MAX > 16 ? 16 : NSTAGE_MAX;
-  static constexpr int NC = NSTAGE / 2;                       // consumer warps, two stages each
+  static constexpr int NP = NSTAGE / 2;                       // consumer groups, two stages each
+  static constexpr int WPU = TP >= 32 ? 2 : 1;                // warps per problem (split by 16-row m-tiles)
+  static constexpr int NC = NP * WPU;                         // consumer warps
   static constexpr int THREADS = 32 * (1 + NC);
   static constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8;
   static_assert(D % 16 == 0 && D >= 32 && D <= 128, "head_dim");
@@ -99,13 +102,13 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], C::WPU);       // every warp of the consumer group releases the stage
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  // problem k of this CTA -> stage (k % NC) * 2 + (k / NC) % 2, consumer k % NC
+  // problem k of this CTA -> stage (k % NP) * 2 + (k / NP) % 2, consumer group k % NP
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -113,8 +116,8 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
       tma_prefetch_desc(&tmV);
       int issued = 0;
       for (int k = 0; k < n_local; ++k) {
-        const int st = (k % C::NC) * 2 + ((k / C::NC) & 1);
-        const int use = k / (2 * C::NC);                    // earlier fills of this stage
+        const int st = (k % C::NP) * 2 + ((k / C::NP) & 1);
+        const int use = k / (2 * C::NP);                    // earlier fills of this stage
         if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, 20)) break;
         const long long u = u_begin + k;
         const int h = (int)(u % p.heads);
@@ -132,25 +135,26 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
         issued = k + 1;
       }
       // drain: the last fill of every stage has landed before the CTA exits
-      for (int k = issued - 2 * C::NC < 0 ? 0 : issued - 2 * C::NC; k < issued; ++k) {
-        const int st = (k % C::NC) * 2 + ((k / C::NC) & 1);
+      for (int k = issued - 2 * C::NP < 0 ? 0 : issued - 2 * C::NP; k < issued; ++k) {
+        const int st = (k % C::NP) * 2 + ((k / C::NP) & 1);
         const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full[st], (k / (2 * C::NC)) & 1))
+        while (!mbar_try_wait(&full[st], (k / (2 * C::NP)) & 1))
           if (globaltimer_ns() - t0 > kWaitLimitNs) { watchdog_trip(21); break; }
       }
     }
     return;
   }
 
-  const int cw = warp - 1;                   // consumer index
+  const int cg = (warp - 1) / C::WPU;       // consumer group
+  const int sub = (warp - 1) % C::WPU;      // this warp's m-tiles: sub, sub + WPU, ...
   const int T = p.T;
   const long long row_stride = (long long)p.HW * p.heads * D;    // elements between frames
   const int n_mt = (T + 15) / 16;
   const int g8 = lane >> 2;                  // fragment row within an 8-row group
   const int q2 = (lane & 3) * 2;             // fragment column pair
-  int j = 0;                                 // this consumer's problem count
-  for (int k = cw; k < n_local; k += C::NC, ++j) {
-    const int st = cw * 2 + (j & 1);
+  int j = 0;                                 // this group's problem count
+  for (int k = cg; k < n_local; k += C::NP, ++j) {
+    const int st = cg * 2 + (j & 1);
     if (!mbar_wait(&full[st], (j >> 1) & 1, 22)) break;
     unsigned char* sb = stages + st * C::STAGE_BYTES;
     const uint32_t aQ = smem_u32(sb), aK = aQ + C::TENSOR_BYTES, aV = aQ + 2 * C::TENSOR_BYTES;
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
     const int s = (int)(bs % p.HW);
     const int b = (int)(bs / p.HW);
 
-    for (int mt = 0; mt < n_mt; ++mt) {
+    for (int mt = sub; mt < n_mt; mt += C::WPU) {
       // ---- S = Q K^T for rows mt*16 .. mt*16+15, all TP key columns
       float sacc[TP / 8][4];
 #pragma unroll
@@ -250,12 +254,15 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
       __syncwarp();
     }
 
-    // ---- write O rows back to their tokens, then hand the stage back
+    // ---- write this warp's O rows back to their tokens, then hand the stage back
     const long long first = (((long long)b * T * p.HW + s) * p.heads + h) * D;   // element of t = 0
-    for (int i = lane; i < T * (D / 8); i += 32) {
-      const int t = i / (D / 8), c = i - t * (D / 8);
-      const uint4 val = *reinterpret_cast<const uint4*>(sb + time_off<D, TP>(t, c));
-      *reinterpret_cast<uint4*>(p.o + first + t * row_stride + c * 8) = val;
+    for (int mt = sub; mt < n_mt; mt += C::WPU) {
+      const int rows = min(16, T - mt * 16);
+      for (int i = lane; i < rows * (D / 8); i += 32) {
+        const int t = mt * 16 + i / (D / 8), c = i % (D / 8);
+        const uint4 val = *reinterpret_cast<const uint4*>(sb + time_off<D, TP>(t, c));
+        *reinterpret_cast<uint4*>(p.o + first + t * row_stride + c * 8) = val;
+      }
     }
     // the stage's next fill is an async-proxy write over these generic-proxy accesses
     fence_proxy_async_smem();

@@ -19,9 +19,12 @@ namespace vdit {
 // so its output is one contiguous span of WC*F elements (F = C*pt*ph*pw).  The
 // CTA first copies the C*pt*ph latent rows those bricks cover (each a
 // contiguous run of WC*pw elements along W) into shared memory, one warp per
-// row with the lanes sweeping the row; then each warp writes whole bricks, the
-// lanes sweeping the brick's F features in order, each feature's source found
-// in a per-CTA table of staged offsets.  No division runs per element.
+// row with 16-byte loads (four in flight per lane) when the row is aligned;
+// then it writes the output span with 16-byte stores, each gathering VEC
+// consecutive features from the staged rows through a per-CTA table of staged
+// offsets.  Staged rows are an odd number of elements apart, so the lanes that
+// gather one brick's channels (one per staged row) fall in different banks.
+// Unaligned shapes take the same path one element at a time.
 
 struct PatchifyShape {
   int N, C, T, H, W, pt, ph, pw;
@@ -36,16 +39,22 @@ constexpr int kPatchifyThreads = 256;
 template <typename E>
 __global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* __restrict__ latent,
                                                                       E* __restrict__ tokens, PatchifyShape s) {
+  constexpr int VEC = 16 / sizeof(E);             // elements per 16-byte vector
   // dynamic shared memory: F staged-row offsets (int), then the staged rows
   int* src_off = reinterpret_cast<int*>(dyn_smem);
   E* rows = reinterpret_cast<E*>(dyn_smem + ((s.F * sizeof(int) + 15) & ~size_t(15)));
   if (watchdog_tripped()) return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int rowlen = s.WC * s.pw;                 // elements per staged row
+  const int rowlen = s.WC * s.pw + ((s.WC * s.pw) % 2 == 0 ? 1 : 0);   // staged row stride (odd)
   const int nrows = s.C * s.pt * s.ph;
   // feature f = ((c*pt + dt)*ph + dh)*pw + dw  reads staged row (c*pt + dt)*ph + dh at dw
   for (int f = threadIdx.x; f < s.F; f += blockDim.x) src_off[f] = (f / s.pw) * rowlen + f % s.pw;
+  // 16-byte paths: every staged row starts 16-byte aligned in global and shared
+  // memory, and every output span does too
+  const bool vec_in = (s.W % VEC) == 0 && ((s.WC * s.pw) % VEC) == 0 &&
+                      (reinterpret_cast<uintptr_t>(latent) & 15) == 0;
+  const bool vec_out = (s.F % VEC) == 0 && (reinterpret_cast<uintptr_t>(tokens) & 15) == 0;
 
   const long long n_jobs = (long long)s.N * s.Tg * s.Hg * s.n_wchunks;
   for (long long job = blockIdx.x; job < n_jobs; job += gridDim.x) {
@@ -69,16 +78,47 @@ __global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* _
       const E* src = latent + ((((long long)n * s.C + c) * s.T + (tq * s.pt + dt)) * s.H + (hq * s.ph + dh)) *
                                   (long long)s.W + (long long)w0 * s.pw;
       E* dst = rows + row * rowlen;
-      for (int x = lane; x < len; x += 32) dst[x] = src[x];
+      if (vec_in) {
+        const int nv = len / VEC;                 // whole 16-byte vectors of the row
+        const uint4* sv = reinterpret_cast<const uint4*>(src);
+        for (int x = lane; x < nv; x += 128) {
+          union { uint4 u; E e[VEC]; } t[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (x + 32 * u < nv) t[u].u = __ldg(sv + x + 32 * u);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (x + 32 * u < nv) {
+#pragma unroll
+              for (int k = 0; k < VEC; ++k) dst[(x + 32 * u) * VEC + k] = t[u].e[k];
+            }
+        }
+        for (int x = nv * VEC + lane; x < len; x += 32) dst[x] = src[x];   // tail shorter than a vector
+      } else {
+        for (int x = lane; x < len; x += 32) dst[x] = src[x];
+      }
     }
     __syncthreads();
 
-    // write the contiguous output span of nb tokens: one warp per brick
+    // write the contiguous output span of nb tokens
     E* out = tokens + (((long long)n * s.Tg + tq) * s.Hg * s.Wg + (long long)hq * s.Wg + w0) * s.F;
-    for (int b = warp; b < nb; b += nwarps) {
-      const E* from = rows + b * s.pw;
-      E* to = out + (long long)b * s.F;
-      for (int f = lane; f < s.F; f += 32) to[f] = from[src_off[f]];
+    if (vec_out) {
+      const int gpb = s.F / VEC;                  // vectors per brick
+      for (int g = threadIdx.x; g < nb * gpb; g += blockDim.x) {
+        const int b = g / gpb;
+        const int f0 = (g - b * gpb) * VEC;
+        const E* from = rows + b * s.pw;
+        union { uint4 u; E e[VEC]; } v;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) v.e[k] = from[src_off[f0 + k]];
+        reinterpret_cast<uint4*>(out)[g] = v.u;
+      }
+    } else {
+      for (int b = warp; b < nb; b += nwarps) {
+        const E* from = rows + b * s.pw;
+        E* to = out + (long long)b * s.F;
+        for (int f = lane; f < s.F; f += 32) to[f] = from[src_off[f]];
+      }
     }
   }
 }

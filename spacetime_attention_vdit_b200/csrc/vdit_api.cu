@@ -248,22 +248,24 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, 
   const int esz = dtype == VDIT_F32 ? 4 : 2;
   const long long brick_bytes = F * esz;
   constexpr long long kStage = 32 * 1024;          // staged latent rows per CTA
-  if (brick_bytes > kStage) return VDIT_ERR_UNSUPPORTED;
+  // shared memory: staged rows (<= 2 * kStage with the padding) + offset table (<= kStage)
+  if (brick_bytes > kStage || F * 4 > kStage) return VDIT_ERR_UNSUPPORTED;
   s.F = (int)F;
   s.WC = (int)std::min<long long>(s.Wg, kStage / brick_bytes);
   s.n_wchunks = (s.Wg + s.WC - 1) / s.WC;
-  const int smem = (int)(((F * 4 + 15) & ~15LL) + (long long)C * pt * ph * s.WC * pw * esz);
+  const long long rowlen = (long long)s.WC * pw + ((s.WC * pw) % 2 == 0 ? 1 : 0);   // odd staged row stride
+  const int smem = (int)(((F * 4 + 15) & ~15LL) + (long long)C * pt * ph * rowlen * esz);
   const long long jobs = (long long)N * s.Tg * s.Hg * s.n_wchunks;
   const long long cap = (long long)sm_count() * 16;
   const unsigned grid = (unsigned)(jobs < cap ? jobs : cap);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   {
-    // staged rows (<= 32 KB) plus the feature offset table (<= 32 KB)
+    // staged rows (<= 32 KB plus one element per row) plus the feature offset table (<= 32 KB)
     static bool done_f[kMaxDevices] = {}, done_b[kMaxDevices] = {};
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
-    if (!ensure_smem(patchify3d_kernel<float>, 2 * kStage + 16, done_f) ||
-        !ensure_smem(patchify3d_kernel<__nv_bfloat16>, 2 * kStage + 16, done_b))
+    if (!ensure_smem(patchify3d_kernel<float>, 3 * kStage + 16, done_f) ||
+        !ensure_smem(patchify3d_kernel<__nv_bfloat16>, 3 * kStage + 16, done_b))
       return VDIT_ERR_CUDA;
   }
   if (dtype == VDIT_F32)

@@ -146,7 +146,8 @@ def test_register_budget_fits_each_sm_subpartition():
         D, TP = int(m.group(1)), int(m.group(2))
         stage = 3 * TP * D * 2
         nstage = min(16, (196608 // stage) & ~1)
-        return 32 * (1 + nstage // 2)
+        wpu = 2 if TP >= 32 else 1
+        return 32 * (1 + (nstage // 2) * wpu)
     assert regs, "no ptxas report"
     for kname, r in regs.items():
         warps = block_of(kname) // 32
