@@ -123,6 +123,67 @@ __global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* _
   }
 }
 
+// The pages' own patch, (1, 2, 2), on float32: each output float4 is one channel
+// of one brick, {row(c, dh = 0)[2b], [2b + 1], row(c, 1)[2b], [2b + 1]}, i.e. two
+// float2 reads from two staged rows - no offset table.  Staged rows are
+// 2*WC + 2 floats apart (8-byte aligned, 2 words mod 32 banks), which keeps the
+// float2 staging stores and the float2 gathers at or near the two-wavefront
+// minimum of a 256-byte warp access.  Output float4 stores are coalesced.
+__global__ void __launch_bounds__(kPatchifyThreads) patchify122_f32_kernel(const float* __restrict__ latent,
+                                                                           float* __restrict__ tokens,
+                                                                           PatchifyShape s) {
+  float* rows = reinterpret_cast<float*>(dyn_smem);
+  if (watchdog_tripped()) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int rs = 2 * s.WC + 2;                    // staged row stride (floats)
+  const int nrows = 2 * s.C;                      // (c, dh)
+  const long long plane = (long long)s.H * s.W;
+  const long long n_jobs = (long long)s.N * s.Tg * s.Hg * s.n_wchunks;
+  for (long long job = blockIdx.x; job < n_jobs; job += gridDim.x) {
+    const int wc = (int)(job % s.n_wchunks);
+    long long r = job / s.n_wchunks;
+    const int hq = (int)(r % s.Hg);
+    r /= s.Hg;
+    const int tq = (int)(r % s.Tg);
+    const int n = (int)(r / s.Tg);
+    const int w0 = wc * s.WC;
+    const int nb = min(s.WC, s.Wg - w0);
+    const int len = 2 * nb;                       // floats of each staged row
+    __syncthreads();
+    for (int row = warp; row < nrows; row += nwarps) {
+      const int c = row >> 1, dh = row & 1;
+      const float* src = latent + (((long long)n * s.C + c) * s.T + tq) * plane + (long long)(2 * hq + dh) * s.W +
+                         2LL * w0;
+      float* dst = rows + row * rs;
+      const int n4 = len >> 2;                    // 16-byte vectors (src is 16-byte aligned, see launcher)
+      const float4* sv = reinterpret_cast<const float4*>(src);
+      for (int x = lane; x < n4; x += 128) {
+        float4 t[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (x + 32 * u < n4) t[u] = __ldg(sv + x + 32 * u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (x + 32 * u < n4) {
+            float2* d = reinterpret_cast<float2*>(dst + 4 * (x + 32 * u));
+            d[0] = make_float2(t[u].x, t[u].y);
+            d[1] = make_float2(t[u].z, t[u].w);
+          }
+      }
+      for (int x = 4 * n4 + lane; x < len; x += 32) dst[x] = src[x];
+    }
+    __syncthreads();
+    float4* out = reinterpret_cast<float4*>(tokens + (((long long)n * s.Tg + tq) * s.Hg * s.Wg +
+                                                      (long long)hq * s.Wg + w0) * s.F);
+    for (int g = threadIdx.x; g < nb * s.C; g += blockDim.x) {
+      const int b = g / s.C, c = g - b * s.C;
+      const float2 a = *reinterpret_cast<const float2*>(rows + (2 * c) * rs + 2 * b);
+      const float2 d = *reinterpret_cast<const float2*>(rows + (2 * c + 1) * rs + 2 * b);
+      out[g] = make_float4(a.x, a.y, d.x, d.y);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // 3D RoPE
 // ---------------------------------------------------------------------------

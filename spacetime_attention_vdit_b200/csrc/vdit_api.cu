@@ -268,7 +268,21 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, 
         !ensure_smem(patchify3d_kernel<__nv_bfloat16>, 3 * kStage + 16, done_b))
       return VDIT_ERR_CUDA;
   }
-  if (dtype == VDIT_F32)
+  // (every staged row must start 16-byte aligned: W a multiple of 4, and each chunk's
+  // first column 2*w0 too, which holds with one chunk or an even chunk width)
+  if (dtype == VDIT_F32 && pt == 1 && ph == 2 && pw == 2 && W % 4 == 0 && (s.n_wchunks == 1 || s.WC % 2 == 0) &&
+      aligned16(latent) && aligned16(tokens)) {
+    // the (1, 2, 2) float32 fast path: 2*C staged rows of 2*WC + 2 floats
+    const int smem122 = (int)(2LL * C * (2LL * s.WC + 2) * 4);
+    if (smem122 > 48 * 1024) {
+      static bool done[kMaxDevices] = {};
+      static std::mutex mu2;
+      std::lock_guard<std::mutex> lock(mu2);
+      if (!ensure_smem(patchify122_f32_kernel, 3 * kStage + 16, done)) return VDIT_ERR_CUDA;
+    }
+    patchify122_f32_kernel<<<grid, kPatchifyThreads, smem122, st>>>(static_cast<const float*>(latent),
+                                                                      static_cast<float*>(tokens), s);
+  } else if (dtype == VDIT_F32)
     patchify3d_kernel<float><<<grid, kPatchifyThreads, smem, st>>>(static_cast<const float*>(latent),
                                                                    static_cast<float*>(tokens), s);
   else

@@ -135,3 +135,15 @@ def test_rope_full_size_sampled(B, grid):
     L = grid[0] * grid[1] * grid[2]
     toks = synthetic.sample_rows(L, 4096, seed=0)
     _rope_check(B, grid, 40, 128, (44, 42, 42), seed=0, tokens=toks)
+
+
+@pytest.mark.parametrize("shape", [(1, 5, 3, 6, 1028), (1, 4, 2, 5, 2056), (2, 3, 2, 4, 12), (1, 16, 2, 4, 8)])
+def test_patchify_122_fast_path_edges(shape):
+    """(1,2,2) float32 shapes that exercise the fast path's chunking: several
+    W-chunks (odd channel count, even chunk width), odd H (a floored row), and
+    rows of a single vector."""
+    import spacetime_attention_vdit_b200 as v
+    lat = synthetic.latent_f32(*shape, seed=2)
+    got = v.patchify_3d(torch.from_numpy(lat).cuda(), (1, 2, 2)).cpu().numpy()
+    exp = ref.patchify(lat, 1, 2, 2)
+    assert np.array_equal(got.view(np.uint32), exp.view(np.uint32))
