@@ -13,9 +13,10 @@
 //   warp 0      TMA producer: Q tiles once; K_j into a K ring and V_j into a
 //               V ring (K is needed one P.V product earlier than V);
 //   warp 1      allocates all 512 TMEM columns and issues every UMMA from one
-//               thread: S_i = Q_i K_j^T (smem x smem) into tile i's score
-//               columns, then O_i += P_i V_j with P_i read from TMEM (the
-//               softmax overwrote tile i's scores with bf16 probabilities);
+//               thread, in a fixed order: O_i += P_i V_j with P_i read from
+//               TMEM (the softmax overwrote tile i's scores with bf16
+//               probabilities), then at once S_i = Q_i K_{j+1}^T (smem x smem)
+//               into the same columns, for tile 0 and then tile 1;
 //   warps 2..5  softmax of query tile 0, warps 6..9 of tile 1, one query row
 //               per thread (TMEM lane = row).
 // The two tiles ping-pong: while one warpgroup exponentiates its scores the
@@ -24,8 +25,9 @@
 //
 // Softmax per tile and row: running max m kept unless a new tile raises it by
 // more than 2^8 (exact rescaling rule: P stays below 2^8 and O/l is unchanged);
-// P = 2^(s * scale * log2e - m) rounded to bf16; O rescaled in TMEM only when m
-// moved; at the end O / l and the row's log-sum-exp are written out.
+// P = 2^(s * scale * log2e - m) rounded to bf16, one pair in kFmaPairEvery
+// exponentiated on the FMA pipe to unload the MUFU; O rescaled in TMEM only
+// when m moved; at the end O / l and the row's log-sum-exp are written out.
 //
 // Each CTA sweeps the key tiles starting at tile (query block mod tiles), so
 // the CTAs of one head, which run together, read different K/V lines from L2
@@ -52,7 +54,7 @@ struct AttnCfg {
   static constexpr int TILE_BYTES = BM * D * 2;
   static constexpr int NK = D >= 128 ? 3 : 4;                  // K ring stages
   static constexpr int NV = D >= 128 ? 2 : (D >= 64 ? 3 : 4);  // V ring stages
-  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 3 * NQ + 1;
+  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NQ + 1;
   static constexpr int SMEM_BYTES = 1024 + (NQ + NK + NV) * TILE_BYTES + NBARS * 8 + 16;
   static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -105,6 +107,50 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int si
   return __all_sync(0xffffffffu, ok) != 0;
 }
 
+// 2^x on the FMA pipe, for x <= 8: x = n + f with n = rint(x) (the 1.5 * 2^23
+// rounding constant) and |f| <= 1/2; 2^f from a cubic fitted here by
+// relative-error least squares on [-1/2, 1/2] (max relative error 7.8e-5, below
+// half a bf16 ulp); n is added to the exponent field.  Below -125 the result is
+// 0, like the MUFU's flushed 2^x there, and a masked score (-inf) gives exactly 0.
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 rnd = make_float2(12582912.f, 12582912.f);
+  const float2 t = fadd2(xc, rnd);                                         // rnd + rint(x)
+  const float2 f = fadd2(xc, ffma2(t, make_float2(-1.f, -1.f), rnd));     // x - rint(x)
+  float2 q = ffma2(make_float2(5.5088737e-2f, 5.5088737e-2f), f, make_float2(0.24260406f, 0.24260406f));
+  q = ffma2(q, f, make_float2(0.69327623f, 0.69327623f));
+  q = ffma2(q, f, make_float2(0.99992894f, 0.99992894f));
+  const float lo = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  const float hi = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return make_float2(x.x < -125.f ? 0.f : lo, x.y < -125.f ? 0.f : hi);
+}
+
+// One score pair in kFmaPairEvery is exponentiated on the FMA pipe (ex2_fma2),
+// the rest on the MUFU: the MUFU alone needs about as many cycles per key tile
+// as the tensor core, so a small share moved off it shortens the softmax.
+constexpr int kFmaPairEvery = 32;
+
+// P = 2^(s * scale_log2 - m) for one row's 128 scores, packed to bf16 pairs and
+// stored over the row's score columns, 16 keys (8 columns) per store so that
+// few packed values are live at once; the packed partial sums go to sp.
+__device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_s, float2 sc2, float2 nm2,
+                                         float2 (&sp)[4]) {
+#pragma unroll
+  for (int h8 = 0; h8 < 8; ++h8) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const int c = h8 >> 1, ee = (h8 & 1) * 16 + e;
+      const float2 x = ffma2(make_float2(__uint_as_float(s[c][ee]), __uint_as_float(s[c][ee + 1])), sc2, nm2);
+      const bool on_fma = ((h8 * 8 + (e >> 1)) % kFmaPairEvery) == kFmaPairEvery - 1;
+      const float2 pr = on_fma ? ex2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      sp[(e >> 1) & 3] = fadd2(sp[(e >> 1) & 3], pr);
+      pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st8(t_s + h8 * 8, pk);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -123,8 +169,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* v_empty = v_full + C::NV;
   uint64_t* s_full = v_empty + C::NV;      // [NQ]
   uint64_t* p_full = s_full + C::NQ;       // [NQ]
-  uint64_t* o_done = p_full + C::NQ;       // [NQ]
-  uint64_t* drain = o_done + C::NQ;
+  uint64_t* drain = p_full + C::NQ;        // every UMMA of the CTA has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -149,7 +194,6 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < C::NQ; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);           // one elected lane per softmax warp
-      mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -237,7 +281,6 @@ __global__ void __launch_bounds__(320, 1)
           umma_ts(tmem + C::O_COL + i * C::BM, tmem + C::S_COL + i * C::BN + kk * 8, b, C::IDESC_PV,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&o_done[i]);
       };
       bool ok = mbar_wait(q_full, 0, kSiteQFull) && mbar_wait(&k_full[0], 0, kSiteKFull);
       if (ok) {
@@ -245,43 +288,31 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < nq; ++i) qk(i, 0);
         umma_commit(&k_empty[0]);
       }
-      // Event loop: issue whichever product is ready, so that while tile i waits
-      // for its P.V to finish (before its scores may be overwritten) the tensor
-      // core works on the other tile.  npv[i] / nqk[i]: next iteration whose
-      // P.V / QK^T tile i issues; a K or V stage is released once both tiles
-      // have issued the products that read it.
-      int npv[2] = {0, nq > 1 ? 0 : n};
-      int nqk[2] = {1, nq > 1 ? 1 : n};
-      int v_rel = 0, k_rel = 1;
-      unsigned long long t_last = globaltimer_ns();
-      while (ok && (npv[0] < n || npv[1] < n)) {
-        bool progress = false;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int jp = npv[i];
-          if (jp < n && nqk[i] > jp && mbar_test(&p_full[i], jp & 1) &&
-              mbar_test(&v_full[jp % C::NV], (jp / C::NV) & 1)) {
-            tc_fence_after();
-            pv(i, jp);
-            npv[i] = jp + 1;
-            progress = true;
-            for (const int lo = min(npv[0], npv[1]); v_rel < lo; ++v_rel) umma_commit(&v_empty[v_rel % C::NV]);
-          }
-          const int jq = nqk[i];
-          if (jq < n && npv[i] >= jq && mbar_test(&o_done[i], (jq - 1) & 1) &&
-              mbar_test(&k_full[jq % C::NK], (jq / C::NK) & 1)) {
-            tc_fence_after();
-            qk(i, jq);
-            nqk[i] = jq + 1;
-            progress = true;
-            for (const int lo = min(nqk[0], nqk[1]); k_rel < lo; ++k_rel) umma_commit(&k_empty[k_rel % C::NK]);
+      // Fixed issue order, the one the two tiles' ping-pong settles into:
+      //   O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T, O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T.
+      // QK^T of a tile follows its P.V at once although it overwrites the
+      // columns P.V reads: the UMMAs one thread issues execute in issue order
+      // (tcgen05 pipelined-instruction ordering), so no wait is needed between
+      // them.  The issuing thread sleeps in each barrier wait rather than
+      // polling, which would take issue slots from the softmax warp sharing its
+      // SM sub-partition.  A K or V stage is released once both tiles have
+      // issued the products that read it.
+      for (int j = 0; j < n && ok; ++j) {
+        for (int i = 0; i < nq; ++i) {
+          if (i == 0) ok = mbar_wait(&v_full[j % C::NV], (j / C::NV) & 1, kSiteVFull);
+          if (ok) ok = mbar_wait(&p_full[i], j & 1, kSitePFull);
+          if (!ok) break;
+          tc_fence_after();
+          pv(i, j);
+          if (j + 1 < n) {
+            if (i == 0) ok = mbar_wait(&k_full[(j + 1) % C::NK], ((j + 1) / C::NK) & 1, kSiteKFull);
+            if (!ok) break;
+            qk(i, j + 1);
           }
         }
-        if (progress) {
-          t_last = globaltimer_ns();
-        } else if (watchdog_tripped() || globaltimer_ns() - t_last > kWaitLimitNs) {
-          watchdog_trip(kSiteODone);
-          ok = false;
+        if (ok) {
+          umma_commit(&v_empty[j % C::NV]);
+          if (j + 1 < n) umma_commit(&k_empty[(j + 1) % C::NK]);
         }
       }
       // every UMMA issued above has finished before TMEM is released
@@ -316,15 +347,13 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
       }
-      float mp[8];                                // eight independent max chains
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four max chains
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mp[e & 7] = fmaxf(mp[e & 7], __uint_as_float(s[c][e]));
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        for (int e = 0; e < 32; e += 2)
+          mp[(e >> 1) & 3] = fmax3(mp[(e >> 1) & 3], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+      const float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]), mp[3]);
       const float m_new = mx * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -339,21 +368,9 @@ __global__ void __launch_bounds__(320, 1)
       const float2 nm2 = make_float2(-m_use, -m_use);
       float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};   // four independent packed sum chains
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), sc2, nm2);
-          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          sp[(e >> 1) & 3] = fadd2(sp[(e >> 1) & 3], pr);
-          pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
-        }
-        // P over this tile's own score columns: keys 32c .. 32c+31 -> 16 columns
-        tmem_st16(t_s + c * 16, pk);
-      }
+      exp_tile(s, t_s, sc2, nm2, sp);     // P over this tile's own score columns
       const float2 s01 = fadd2(fadd2(sp[0], sp[1]), fadd2(sp[2], sp[3]));
-      const float rsum = s01.x + s01.y;
+      l_sum = l_sum * alpha + (s01.x + s01.y);
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -365,7 +382,6 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32(t_o + c * 32, o);
         }
       }
-      l_sum = l_sum * alpha + rsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -373,7 +389,7 @@ __global__ void __launch_bounds__(320, 1)
     }
 
     // ------------------------------------------------------------- epilogue
-    if (ok && warp_wait(&o_done[tile], (n - 1) & 1, kSiteODone)) {
+    if (ok && warp_wait(drain, 0, kSiteODone)) {
       tc_fence_after();
       const int i = q0 + tile * C::BM + row;      // position in the sequence
       const float inv_l = 1.f / l_sum;

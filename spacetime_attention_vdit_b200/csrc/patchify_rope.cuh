@@ -35,6 +35,11 @@ struct PatchifyShape {
 };
 
 constexpr int kPatchifyThreads = 256;
+// The (1, 2, 2) float32 path runs small CTAs, many per SM, so that one CTA's
+// loads overlap another's stores; each job keeps a whole latent row, since
+// shorter contiguous runs cost more than the lost occupancy.
+constexpr int kPatchify122Threads = 128;
+constexpr int kPatchify122CtasPerSm = 32;
 
 template <typename E>
 __global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* __restrict__ latent,
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(kPatchifyThreads) patchify3d_kernel(const E* _
 // 2*WC + 2 floats apart (8-byte aligned, 2 words mod 32 banks), which keeps the
 // float2 staging stores and the float2 gathers at or near the two-wavefront
 // minimum of a 256-byte warp access.  Output float4 stores are coalesced.
-__global__ void __launch_bounds__(kPatchifyThreads) patchify122_f32_kernel(const float* __restrict__ latent,
+__global__ void __launch_bounds__(kPatchify122Threads) patchify122_f32_kernel(const float* __restrict__ latent,
                                                                            float* __restrict__ tokens,
                                                                            PatchifyShape s) {
   float* rows = reinterpret_cast<float*>(dyn_smem);

@@ -93,13 +93,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up after
-// kWaitLimitNs, or at once if another wait anywhere on the device gave up, and
-// then records `site` in the watchdog and returns false.
+// kWaitLimitNs, or soon after another wait anywhere on the device gave up, and
+// then records `site` in the watchdog and returns false.  The clock and the
+// device-wide flag are read only between runs of 64 try_waits: each read costs
+// hundreds of cycles, during which a completed phase would go unnoticed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
+  for (int spin = 0; spin < 64; ++spin)
+    if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    for (int spin = 0; spin < 64; ++spin)
+      if (mbar_try_wait(bar, parity)) return true;
     if (watchdog_tripped() || globaltimer_ns() - t0 > kWaitLimitNs) {
       watchdog_trip(site);
       return false;
@@ -205,6 +209,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 32 lanes x 8 columns of 32-bit from registers.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // 32 lanes x 16 columns of 32-bit from registers.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -286,6 +297,13 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "=l"(d)
       : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
   return *reinterpret_cast<float2*>(&d);
+}
+
+// max(a, b, c) in one instruction (three-operand form, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

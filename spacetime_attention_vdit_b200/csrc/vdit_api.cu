@@ -274,13 +274,15 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, 
       aligned16(latent) && aligned16(tokens)) {
     // the (1, 2, 2) float32 fast path: 2*C staged rows of 2*WC + 2 floats
     const int smem122 = (int)(2LL * C * (2LL * s.WC + 2) * 4);
+    const long long cap122 = (long long)sm_count() * kPatchify122CtasPerSm;
+    const unsigned grid122 = (unsigned)(jobs < cap122 ? jobs : cap122);
     if (smem122 > 48 * 1024) {
       static bool done[kMaxDevices] = {};
       static std::mutex mu2;
       std::lock_guard<std::mutex> lock(mu2);
       if (!ensure_smem(patchify122_f32_kernel, 3 * kStage + 16, done)) return VDIT_ERR_CUDA;
     }
-    patchify122_f32_kernel<<<grid, kPatchifyThreads, smem122, st>>>(static_cast<const float*>(latent),
+    patchify122_f32_kernel<<<grid122, kPatchify122Threads, smem122, st>>>(static_cast<const float*>(latent),
                                                                       static_cast<float*>(tokens), s);
   } else if (dtype == VDIT_F32)
     patchify3d_kernel<float><<<grid, kPatchifyThreads, smem, st>>>(static_cast<const float*>(latent),

@@ -137,7 +137,7 @@ def test_register_budget_fits_each_sm_subpartition():
         if m and name:
             regs[name] = int(m.group(1))
     threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256,
-               "patchify122_f32_kernel": 256}
+               "patchify122_f32_kernel": 128}
 
     def block_of(kname):
         for key, t in threads.items():
