@@ -418,6 +418,12 @@ def main():
         if n == "attn_space":
             r["tflops"] = space_f / (per_row[n] * 1e-3) / 1e12
         rows[n] = r
+    # divided attention against full attention: the pages' count of attended
+    # pairs, L^2 / (HW*T^2 + T*HW^2) (20.88 at 720p), beside the measured time ratio
+    pairs_full = d["L"] * d["L"]
+    pairs_div = d["HW"] * d["Tg"] * d["Tg"] + d["Tg"] * d["HW"] * d["HW"]
+    divided = {"pair_ratio": pairs_full / pairs_div,
+               "time_ratio": per_row["attn_full"] / (per_row["attn_time"] + per_row["attn_space"])}
 
     # ---- auxiliary: patchify at a size where bandwidth, not launch latency, shows
     aux = None
@@ -460,6 +466,7 @@ def main():
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "aux": aux,
+                "divided_vs_full": divided,
                 "frac_of_nominal_dense_bf16": achieved / 2250.0}
         print(json.dumps(line), flush=True)
     if world > 1:
