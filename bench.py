@@ -42,6 +42,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "attention TFLOP/s and ms/layer at 32,760 tokens; % of B200 dense BF16 peak"
 
+TEXT_TOKENS = 512          # prompt tokens the video tokens cross-attend to (towardsai section 5)
+
 WORKLOADS = {
     # name: (B, T latent frames, H latent, W latent, heads, head_dim, description)
     "480p81_cfg_pair": (2, 21, 60, 104, 40, 128,
@@ -447,6 +449,30 @@ def main():
                                           "bytes": pbytes}}
         del big, big_tok
 
+    # ---- next row: text cross-attention, the video tokens of this workload against
+    # 512 prompt tokens (towardsai section 5, Sub-Layer 2); timed on its own
+    cross = None
+    if not args.no_aux:
+        Lk = TEXT_TOKENS
+        kt = torch.empty((d["B"], Lk, Hh, D), dtype=torch.bfloat16, device=dev).normal_()
+        vt = torch.empty_like(kt).normal_()
+        oc = torch.empty_like(q)
+        for _ in range(3):
+            vd.attn_cross(q, kt, vt, out=oc)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        a.record(stream)
+        for _ in range(reps):
+            vd.attn_cross(q, kt, vt, out=oc)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        cms = a.elapsed_time(b_) / reps
+        cflops = 4.0 * d["B"] * Hh * L * Lk * D
+        cross = {"attn_cross_512": {"Lq": L, "Lk": Lk, "ms": cms, "tflops": cflops / (cms * 1e-3) / 1e12,
+                                    "frac_of_sustained": cflops / (cms * 1e-3) / 1e12
+                                    / peaks["bf16_tflops_sustained"]}}
+        del kt, vt, oc
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, s, desc = oracle_sample(d, 15.0)
@@ -466,7 +492,7 @@ def main():
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clocks, "aux": aux,
-                "divided_vs_full": divided,
+                "divided_vs_full": divided, "next_rows": cross,
                 "frac_of_nominal_dense_bf16": achieved / 2250.0}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -13,11 +13,15 @@
  *        or
  *        vdit_attn_divided_time  attention over the T tokens at each spatial site
  *        vdit_attn_divided_space attention over the H'*W' tokens of each frame
+ *     -> vdit_attn_cross         the video tokens attend to the text tokens' keys
+ *                                and values (the block's second attention)
  *
  * Sources (page title, section):
  *   [towardsai]  "How AI Generates Video: Inside Sora and Wan2.1 on a Real GPU",
  *                sections 4 (spacetime tubes, 3D factorized RoPE), 5 (full 3D
- *                self-attention) and 7 (the [7800 x 7800] matrix, token order).
+ *                self-attention; "Sub-Layer 2", text cross-attention against
+ *                512 prompt tokens) and 7 (the [7800 x 7800] matrix, token
+ *                order).
  *   [cheatsheet] "Video and 3D Generation" (aiengineeringfromscratch.com):
  *                "Formulas and numbers" (video tokens, divided attention),
  *                "Tiny video DiT" (Conv3d patchify, time pass then space pass),
@@ -167,6 +171,23 @@ int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o,
 int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int T, int HW, int heads, int head_dim, float scale,
                             vdit_stream_t stream);
+
+/*
+ * vdit_attn_cross - text cross-attention [towardsai s.5, "Sub-Layer 2": the
+ * video tokens supply the queries, the text prompt's tokens the keys and
+ * values; aicassindra "Step 3": every block also reads the text embeddings].
+ *
+ *   O[b, i, h, :] = sum_j softmax_j(scale * Q[b,i,h,:] . K[b,j,h,:]) V[b, j, h, :]
+ *
+ * with i over the Lq query tokens and j over the Lk key tokens; non-causal, no
+ * mask (a caller that pads the prompt passes only the tokens to attend to).
+ * q, o: [B, Lq, heads, head_dim]; k, v: [B, Lk, heads, head_dim]; lse: NULL or
+ * [B, heads, Lq].  No positions are applied (text tokens carry none).
+ * Numerics, alignment and errors as for vdit_attn_full.
+ */
+int vdit_attn_cross(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int Lq, int Lk, int heads, int head_dim, float scale,
+                    vdit_stream_t stream);
 
 /* Text for a status code (static storage; never NULL). */
 const char* vdit_status_string(int status);

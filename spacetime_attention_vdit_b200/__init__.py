@@ -50,6 +50,7 @@ _SIGNATURES = {
     "vdit_attn_full": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_time": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_space": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
+    "vdit_attn_cross": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_device_status": [ctypes.POINTER(ctypes.c_uint)],
     "vdit_version": [],
 }
@@ -153,9 +154,12 @@ def rope_3d(q: torch.Tensor, k: torch.Tensor, grid, split=None, theta: float = 1
     return q_out, k_out
 
 
-def _attn_io(q, k, v, out, lse):
-    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
-        raise ValueError("q, k and v must all be [B, L, heads, head_dim]")
+def _attn_io(q, k, v, out, lse, cross=False):
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q, k and v must be [B, L, heads, head_dim], k and v of one shape")
+    if (q.shape != k.shape) if not cross else (q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]):
+        raise ValueError("q and k must agree in batch, heads and head_dim" if cross
+                         else "q, k and v must all be [B, L, heads, head_dim]")
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n, torch.bfloat16)
     if out is None:
@@ -181,6 +185,18 @@ def attn_full(q, k, v, out=None, lse=None, scale: float = 0.0, stream=None):
     B, L, Hh, D = q.shape
     _check("vdit_attn_full", lib().vdit_attn_full(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, L, Hh, D,
+        float(scale), _stream(stream)))
+    return out if lse_t is None else (out, lse_t)
+
+
+def attn_cross(q, k, v, out=None, lse=None, scale: float = 0.0, stream=None):
+    """Cross-attention: q [B, Lq, heads, D] over k, v [B, Lk, heads, D] (the video
+    tokens attending to the text tokens).  ``lse=True`` also returns [B, heads, Lq]."""
+    out, lse_t, lse_p = _attn_io(q, k, v, out, lse, cross=True)
+    B, Lq, Hh, D = q.shape
+    Lk = k.shape[1]
+    _check("vdit_attn_cross", lib().vdit_attn_cross(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, Lq, Lk, Hh, D,
         float(scale), _stream(stream)))
     return out if lse_t is None else (out, lse_t)
 

@@ -77,12 +77,13 @@ struct AttnParams {
   __nv_bfloat16* o;
   float* lse;          // may be null
   int n_seq;           // sequences
-  int L;               // tokens per sequence
+  int L;               // query tokens per sequence
+  int Lk;              // key tokens per sequence (= L except for cross-attention)
   int heads;
   int grp;             // see AttnMode
   int mode;
   int n_qblocks;       // ceil(L / 256): CTAs per (sequence, head)
-  int n_kv;            // ceil(L / 128)
+  int n_kv;            // ceil(Lk / 128)
   float scale_log2;    // scale * log2(e)
 };
 
@@ -339,7 +340,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, s[c]);
       tmem_ld_wait();
 
-      const int valid = p.L - ((j + j0) % n) * C::BN;   // keys of this tile inside the sequence
+      const int valid = p.Lk - ((j + j0) % n) * C::BN;  // keys of this tile inside the sequence
       if (valid < C::BN) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)

@@ -96,7 +96,7 @@ bool make_qkv_map(CUtensorMap* map, const void* base, int D, int heads, long lon
 
 template <int D>
 int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq, int L,
-                   int grp, int heads, float scale, cudaStream_t stream) {
+                   int Lk, int grp, int heads, float scale, cudaStream_t stream) {
   using C = AttnCfg<D>;
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
@@ -122,21 +122,26 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
     pos_stride = tok;
     batch_stride = tok * L;
   }
+  // keys and values: the same view, with Lk positions per sequence when they
+  // come from another token array (cross-attention; kSeq only)
+  const long long k_positions = mode == kTime ? positions : Lk;
+  const long long k_batch_stride = mode == kTime ? batch_stride : tok * Lk;
   CUtensorMap mq, mk, mv;
   if (!make_qkv_map(&mq, q, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride) ||
-      !make_qkv_map(&mk, k, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride) ||
-      !make_qkv_map(&mv, v, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride))
+      !make_qkv_map(&mk, k, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride) ||
+      !make_qkv_map(&mv, v, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride))
     return VDIT_ERR_CUDA;
   AttnParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.n_seq = n_seq;
   p.L = L;
+  p.Lk = mode == kTime ? L : Lk;
   p.heads = heads;
   p.grp = grp;
   p.mode = mode;
   p.n_qblocks = (L + C::NQ * C::BM - 1) / (C::NQ * C::BM);
-  p.n_kv = (L + C::BN - 1) / C::BN;
+  p.n_kv = (p.Lk + C::BN - 1) / C::BN;
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = (long long)n_seq * heads * p.n_qblocks;
   if (grid > 0x7fffffffLL) return VDIT_ERR_SHAPE;
@@ -145,11 +150,11 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
 }
 
 int dispatch_tcgen05(int D, const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq,
-                     int L, int grp, int heads, float scale, cudaStream_t stream) {
+                     int L, int Lk, int grp, int heads, float scale, cudaStream_t stream) {
   switch (D) {
-    case 32: return launch_tcgen05<32>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
-    case 64: return launch_tcgen05<64>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
-    case 128: return launch_tcgen05<128>(q, k, v, o, lse, mode, n_seq, L, grp, heads, scale, stream);
+    case 32: return launch_tcgen05<32>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
+    case 64: return launch_tcgen05<64>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
+    case 128: return launch_tcgen05<128>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
     default: return VDIT_ERR_UNSUPPORTED;
   }
 }
@@ -322,7 +327,16 @@ int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* 
                    int head_dim, float scale, vdit_stream_t stream) {
   const int rc = check_attn_args(q, k, v, o, lse, B, L, heads, head_dim);
   if (rc != VDIT_OK) return rc;
-  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, L, 1, heads, resolve_scale(scale, head_dim),
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, L, L, 1, heads, resolve_scale(scale, head_dim),
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vdit_attn_cross(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq, int Lk,
+                    int heads, int head_dim, float scale, vdit_stream_t stream) {
+  int rc = check_attn_args(q, k, v, o, lse, B, Lq, heads, head_dim);
+  if (rc == VDIT_OK) rc = check_attn_args(q, k, v, o, lse, B, Lk, heads, head_dim);
+  if (rc != VDIT_OK) return rc;
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, Lq, Lk, 1, heads, resolve_scale(scale, head_dim),
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -332,7 +346,7 @@ int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o
   const int rc = check_attn_args(q, k, v, o, lse, (long long)B * T, HW, heads, head_dim);
   if (rc != VDIT_OK) return rc;
   if ((long long)B * T > 0x7fffffffLL) return VDIT_ERR_SHAPE;
-  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B * T, HW, T, heads, resolve_scale(scale, head_dim),
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B * T, HW, HW, T, heads, resolve_scale(scale, head_dim),
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -345,7 +359,7 @@ int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o,
   const float sc = resolve_scale(scale, head_dim);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T > 64)  // long clips: the tensor-core kernel over a strided view, one sequence per site
-    return dispatch_tcgen05(head_dim, q, k, v, o, lse, kTime, B * HW, T, HW, heads, sc, st);
+    return dispatch_tcgen05(head_dim, q, k, v, o, lse, kTime, B * HW, T, T, HW, heads, sc, st);
   TimeParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;

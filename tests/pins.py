@@ -227,7 +227,23 @@ def pin_attention_special(attention):
     assert np.allclose(np.exp(s - lse[0, 0][:, None]).sum(axis=1), 1.0, atol=1e-13)
 
 
-ATTENTION_PINS = [pin_attention_sdpa, pin_attention_brute, pin_attention_special]
+def pin_attention_cross(attention):
+    """Cross-attention (towardsai section 5, Sub-Layer 2: the video tokens supply
+    the queries, the text tokens the keys and values): Lq != Lk, against torch
+    sdpa in float64 and brute force, with more queries than keys and fewer."""
+    g = np.random.default_rng(34)
+    for Lq, Lk in ((37, 11), (5, 23)):
+        q = g.standard_normal((2, Lq, 2, 16)) * 2.0
+        k, v = (g.standard_normal((2, Lk, 2, 16)) for _ in range(2))
+        o, lse = attention(q, k, v, None)
+        assert o.shape == (2, Lq, 2, 16) and lse.shape == (2, 2, Lq)
+        assert np.allclose(o, _sdpa(q, k, v, 0.25), atol=1e-12)
+        bo, bl = brute.attention(q[1, :, 1].tolist(), k[1, :, 1].tolist(), v[1, :, 1].tolist(), 0.25)
+        assert np.allclose(o[1, :, 1], bo, atol=1e-13)
+        assert np.allclose(lse[1, 1], bl, atol=1e-13)
+
+
+ATTENTION_PINS = [pin_attention_sdpa, pin_attention_brute, pin_attention_special, pin_attention_cross]
 
 # ----------------------------------------------------------------------------
 # Divided attention  (cheatsheet "Tiny video DiT"; "Video as a 3D signal",

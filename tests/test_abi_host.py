@@ -84,7 +84,8 @@ def attn(L, fn="vdit_attn_full", q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, dims=
 
 @pytest.mark.parametrize("fn,dims", [("vdit_attn_full", (1, 256, 2, 128)),
                                      ("vdit_attn_divided_time", (1, 8, 64, 2, 32)),
-                                     ("vdit_attn_divided_space", (1, 8, 64, 2, 32))])
+                                     ("vdit_attn_divided_space", (1, 8, 64, 2, 32)),
+                                     ("vdit_attn_cross", (1, 256, 77, 2, 128))])
 def test_attention_validation(L, fn, dims):
     assert attn(L, fn, dims=dims, q=None) == NULL
     assert attn(L, fn, dims=dims, o=None) == NULL
@@ -96,6 +97,11 @@ def test_attention_validation(L, fn, dims):
     assert attn(L, fn, dims=zero) == SHAPE
     neg = dims[:1] + (-5,) + dims[2:]
     assert attn(L, fn, dims=neg) == SHAPE
+
+
+def test_cross_key_length_checked(L):
+    assert attn(L, "vdit_attn_cross", dims=(1, 256, 0, 2, 128)) == SHAPE
+    assert attn(L, "vdit_attn_cross", dims=(1, 256, -3, 2, 128)) == SHAPE
 
 
 def test_binding_refuses_cpu_tensors(L):

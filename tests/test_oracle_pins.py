@@ -99,6 +99,18 @@ def _rope_variant(x, grid, split, theta=10000.0, freq_width=None, pairing="adjac
     return out
 
 
+def attention_keys_cut_to_queries(q, k, v, scale):
+    """Mistake: the key loop runs over the query length (a self-attention
+    assumption that breaks cross-attention)."""
+    Lq, Lk = q.shape[1], k.shape[1]
+    n = min(Lq, Lk)
+    return ref.attention(q, k[:, :n], v[:, :n], scale)
+
+
+def test_cross_attention_mistake_caught():
+    assert _fails([pins.pin_attention_cross], attention_keys_cut_to_queries) == 1
+
+
 @pytest.mark.parametrize("kw", [
     dict(freq_width=128),            # frequencies from the head width, not the axis width
     dict(pairing="half"),            # rotate-half pairs instead of adjacent pairs
@@ -119,7 +131,7 @@ def _attention_variant(q, k, v, scale, no_scale=False, no_norm=False, drop_last_
         scale = 1.0 / np.sqrt(D)
     if no_scale:
         scale = 1.0
-    o = np.empty_like(v)
+    o = np.empty((B, L, H, v.shape[-1]))
     lse = np.empty((B, H, L))
     for b in range(B):
         for h in range(H):
