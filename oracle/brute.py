@@ -61,3 +61,10 @@ def attention(q, k, v, scale):
         out.append([sum(p[j] * v[j][d] for j in range(len(k))) / z for d in range(len(v[0]))])
         lse.append(m + math.log(z))
     return out, lse
+
+
+def rms_norm(x, weight, eps):
+    """One group: list of floats -> x / sqrt(mean of squares + eps) * weight."""
+    ms = sum(a * a for a in x) / len(x)
+    r = math.sqrt(ms + eps)
+    return [a / r * w for a, w in zip(x, weight)]

@@ -29,6 +29,12 @@ Sources (page title, section):
   and numbers"; "Video as a 3D signal", "Patches and attention" (a time pass
   over the T tokens at each spatial site, a space pass over the HW tokens of
   each frame).
+* Q/K normalisation - towardsai section 5, "Sub-Layer 1": the projected Q and
+  K are RMS-normalised, then rotated by the 3D RoPE.  RMSNorm here is the
+  textbook one: each group of G consecutive channels of a token is divided by
+  sqrt(mean of its squares + eps) and multiplied by a per-channel weight.  The
+  page names neither the group nor eps: G is an argument (head_dim: per head;
+  heads*head_dim: the token's whole projected vector).
 """
 from __future__ import annotations
 
@@ -127,6 +133,29 @@ def rope_3d(x: np.ndarray, grid, split, theta: float = 10000.0, tokens=None) -> 
     out[..., 0::2] = x0 * c - x1 * s
     out[..., 1::2] = x0 * s + x1 * c
     return out
+
+
+def rms_norm(x: np.ndarray, group: int, weight=None, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm of ``[B, L, heads, D]`` in float64 over groups of ``group``
+    consecutive channels of each token's heads*D channels:
+    y = x / sqrt(mean(x^2 over the group) + eps) * weight[channel mod group]."""
+    x = np.asarray(x, dtype=np.float64)
+    B, L, Hh, D = x.shape
+    if group <= 0 or (Hh * D) % group != 0:
+        raise ValueError("group must divide heads * head_dim")
+    w = np.ones(group) if weight is None else np.asarray(weight, dtype=np.float64)
+    if w.shape != (group,):
+        raise ValueError("weight must have one entry per channel of a group")
+    g = x.reshape(B, L, (Hh * D) // group, group)
+    ms = (g * g).mean(axis=-1, keepdims=True)
+    return (g / np.sqrt(ms + eps) * w).reshape(B, L, Hh, D)
+
+
+def qk_norm_rope_3d(x: np.ndarray, grid, split, group: int, weight=None, eps: float = 1e-6,
+                    theta: float = 10000.0, tokens=None) -> np.ndarray:
+    """RMSNorm (``rms_norm``) then the 3D rotation (``rope_3d``), both in float64:
+    what attn1 does to Q and to K before the scores (towardsai section 5)."""
+    return rope_3d(rms_norm(x, group, weight, eps), grid, split, theta, tokens)
 
 
 def rope_3d_fp32(x32: np.ndarray, grid, split, theta: float = 10000.0, tokens=None) -> np.ndarray:

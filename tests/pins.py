@@ -176,6 +176,58 @@ ROPE_PINS = [pin_rope_onehot, pin_rope_complex, pin_rope_relative, pin_rope_norm
              pin_rope_brute]
 
 # ----------------------------------------------------------------------------
+# Q/K RMSNorm before the 3D RoPE  (towardsai section 5, Sub-Layer 1)
+# ----------------------------------------------------------------------------
+
+
+def pin_norm_torch(qk_norm_rope):
+    """With the rotation switched off (all positions 0: a (1,1,1) grid), the
+    result is torch's own rms_norm in float64, per head and per token."""
+    g = np.random.default_rng(41)
+    x = g.standard_normal((2, 1, 3, 16)) * 3.0
+    for group in (16, 48):
+        w = g.standard_normal(group)
+        for eps in (1e-6, 0.5):
+            got = qk_norm_rope(x, (1, 1, 1), (6, 4, 6), group, w, eps)
+            t = torch.from_numpy(x.reshape(2, 1, 48 // group, group))
+            exp = torch.nn.functional.rms_norm(t, (group,), torch.from_numpy(w), eps).numpy().reshape(x.shape)
+            assert np.allclose(got, exp, atol=1e-12, rtol=1e-12)
+
+
+def pin_norm_closed(qk_norm_rope):
+    """A constant group c gives c / sqrt(c^2 + eps) * w; with eps = 0 and w = 1
+    every group has mean square 1 and scaling x does not change the result."""
+    x = np.full((1, 1, 2, 8), 3.0)
+    w = np.arange(1, 9, dtype=np.float64)
+    got = qk_norm_rope(x, (1, 1, 1), (4, 2, 2), 8, w, 0.25)
+    assert np.allclose(got[0, 0, 0], 3.0 / math.sqrt(9.25) * w, atol=1e-14)
+    g = np.random.default_rng(42)
+    x = g.standard_normal((1, 4, 2, 8))
+    y = qk_norm_rope(x, (1, 2, 2), (4, 2, 2), 16, None, 0.0)
+    assert np.allclose((y.reshape(1, 4, 16) ** 2).mean(axis=-1), 1.0, atol=1e-13)
+    assert np.allclose(qk_norm_rope(7.5 * x, (1, 2, 2), (4, 2, 2), 16, None, 0.0), y, atol=1e-13)
+
+
+def pin_norm_brute(qk_norm_rope):
+    """Scalar loops in the page's order: normalise the group, then rotate each
+    head's pairs (brute.rope_vector), with weights that do not commute with the
+    rotation."""
+    g = np.random.default_rng(43)
+    grid, split = (2, 3, 2), (4, 2, 2)
+    x = g.standard_normal((1, 12, 2, 8))
+    w = g.standard_normal(16) + 2.0
+    got = qk_norm_rope(x, grid, split, 16, w, 1e-3)
+    for l in range(12):
+        pos = (l // 6, (l // 2) % 3, l % 2)
+        y = brute.rms_norm(list(x[0, l].reshape(16)), list(w), 1e-3)
+        for hh in range(2):
+            exp = brute.rope_vector(y[hh * 8:(hh + 1) * 8], pos, split)
+            assert np.allclose(got[0, l, hh], exp, atol=1e-13)
+
+
+NORM_PINS = [pin_norm_torch, pin_norm_closed, pin_norm_brute]
+
+# ----------------------------------------------------------------------------
 # Attention  (towardsai sections 5 and 7)
 # ----------------------------------------------------------------------------
 

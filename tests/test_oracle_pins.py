@@ -27,6 +27,11 @@ def test_attention_pins(pin):
     pin(lambda q, k, v, scale: ref.attention(q, k, v, scale))
 
 
+@pytest.mark.parametrize("pin", pins.NORM_PINS, ids=lambda p: p.__name__)
+def test_norm_pins(pin):
+    pin(ref.qk_norm_rope_3d)
+
+
 def test_divided_pins():
     pins.pin_divided_time(ref.divided_time)
     pins.pin_divided_space(ref.divided_space)
@@ -161,3 +166,32 @@ def test_divided_mistakes_caught():
         pins.pin_divided_time(lambda q, k, v, T, HW, s: ref.divided_space(q, k, v, T, HW, s))
     with pytest.raises(AssertionError):
         pins.pin_divided_space(lambda q, k, v, T, HW, s: ref.divided_time(q, k, v, T, HW, s))
+
+
+# ---- Q/K RMSNorm + RoPE: planted mistakes
+
+
+def _norm_variant(x, grid, split, group, weight=None, eps=1e-6, rope_first=False, eps_outside=False,
+                  sum_not_mean=False, per_head_group=False):
+    x = np.asarray(x, dtype=np.float64)
+    B, L, H, D = x.shape
+    gsz = D if per_head_group else group
+    w = np.ones(group) if weight is None else np.asarray(weight, dtype=np.float64)
+    if gsz != group:
+        w = np.resize(w, gsz)
+    y = ref.rope_3d(x, grid, split) if rope_first else x
+    g = y.reshape(B, L, (H * D) // gsz, gsz)
+    ms = (g * g).sum(axis=-1, keepdims=True) if sum_not_mean else (g * g).mean(axis=-1, keepdims=True)
+    r = (np.sqrt(ms) + eps) if eps_outside else np.sqrt(ms + eps)
+    y = (g / r * w).reshape(B, L, H, D)
+    return y if rope_first else ref.rope_3d(y, grid, split)
+
+
+@pytest.mark.parametrize("kw", [dict(rope_first=True), dict(eps_outside=True), dict(sum_not_mean=True),
+                                dict(per_head_group=True)],
+                         ids=["rope-before-norm", "eps-outside-sqrt", "sum-not-mean", "group-per-head"])
+def test_norm_mistakes_caught(kw):
+    for pin in pins.NORM_PINS:
+        pin(_norm_variant)
+    bad = lambda *a, **k: _norm_variant(*a, **k, **kw)
+    assert _fails(pins.NORM_PINS, bad) >= 1
