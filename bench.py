@@ -514,6 +514,22 @@ def main():
                                     "frac_of_sustained": cflops / (cms * 1e-3) / 1e12
                                     / peaks["bf16_tflops_sustained"]}}
         del kt, vt, oc
+        # next row: Q/K RMSNorm fused with the 3D RoPE (towardsai section 5,
+        # Sub-Layer 1), over each token's whole heads*D vector, weights 1
+        qn, kn = torch.empty_like(q), torch.empty_like(k)
+        width = Hh * D
+        for _ in range(3):
+            vd.qk_norm_rope_3d(q, k, grid, width, q_out=qn, k_out=kn)
+        a.record(stream)
+        for _ in range(reps):
+            vd.qk_norm_rope_3d(q, k, grid, width, q_out=qn, k_out=kn)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        nms = a.elapsed_time(b_) / reps
+        nbytes = 4 * q.numel() * 2
+        cross["qk_norm_rope"] = {"norm_group": width, "ms": nms, "gb_s": nbytes / (nms * 1e-3) / 1e9,
+                                 "frac_hbm": nbytes / (nms * 1e-3) / 1e9 / peaks["hbm_gbs"], "bytes": nbytes}
+        del qn, kn
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

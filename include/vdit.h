@@ -9,6 +9,7 @@
  *     -> vdit_patchify_3d        cut into (pt, ph, pw) spacetime bricks, one token each
  *     -> (projection to per-head Q, K, V: done by the caller)
  *     -> vdit_rope_3d            factorised 3D rotary positions on Q and K
+ *        (or vdit_qk_norm_rope_3d: RMSNorm of Q and K, then the same rotation)
  *     -> vdit_attn_full          full 3D self-attention over all T*H'*W' tokens
  *        or
  *        vdit_attn_divided_time  attention over the T tokens at each spatial site
@@ -127,6 +128,30 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
 int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
                  int B, int Tg, int Hg, int Wg, int heads, int head_dim,
                  int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
+
+/*
+ * vdit_qk_norm_rope_3d - RMSNorm of Q and K, then the 3D RoPE, in one pass
+ * [towardsai s.5, "Sub-Layer 1": the projected Q and K are RMS-normalised, then
+ * rotated with the 3D factorized RoPE].
+ *
+ * Each group of `norm_group` consecutive channels of a token's heads*head_dim
+ * channels (head_dim: per head; heads*head_dim: the token's whole vector) is
+ *   y = x / sqrt(mean(x^2 over the group) + eps) * w[channel mod norm_group],
+ * then rotated exactly as vdit_rope_3d does (same grid, split and theta),
+ * float32 throughout and rounded once to bfloat16 (nearest even).
+ * wq, wk: NULL (weight 1) or device float32 [norm_group], 16-byte aligned.
+ * Layouts, aliasing and the RoPE arguments as for vdit_rope_3d.
+ * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE (also: norm_group not dividing
+ * heads*head_dim, eps negative or not finite), VDIT_ERR_ALIGN,
+ * VDIT_ERR_UNSUPPORTED (norm_group not a multiple of 8; a group other than the
+ * whole token whose 16-byte vectors, norm_group/8, do not divide 32;
+ * heads*head_dim above 8,192; Tg*d_t/2 + Hg*d_h/2 + Wg*d_w/2 above 8,192),
+ * VDIT_ERR_CUDA.
+ */
+int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                         const float* wq, const float* wk, int norm_group, float eps,
+                         int B, int Tg, int Hg, int Wg, int heads, int head_dim,
+                         int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
 
 /*
  * vdit_attn_full - full 3D self-attention [towardsai s.5: every token attends

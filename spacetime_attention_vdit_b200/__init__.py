@@ -48,6 +48,7 @@ _SIGNATURES = {
     "vdit_patchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_rope_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_full": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P],
+    "vdit_qk_norm_rope_3d": [_P, _P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_time": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_space": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_cross": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
@@ -151,6 +152,39 @@ def rope_3d(q: torch.Tensor, k: torch.Tensor, grid, split=None, theta: float = 1
     _check("vdit_rope_3d", lib().vdit_rope_3d(
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
         _dev(k_out, "k_out", torch.bfloat16), B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
+    return q_out, k_out
+
+
+def qk_norm_rope_3d(q: torch.Tensor, k: torch.Tensor, grid, norm_group: int, wq=None, wk=None,
+                    eps: float = 1e-6, split=None, theta: float = 10000.0, q_out=None, k_out=None,
+                    inplace: bool = False, stream=None):
+    """RMSNorm of Q and K over groups of ``norm_group`` channels of each token
+    (head_dim: per head; heads*head_dim: the whole token), weights ``wq``/``wk``
+    (float32 [norm_group] on the device, or None for 1), then the 3D rotation of
+    :func:`rope_3d`, in one pass.  Returns (q_out, k_out)."""
+    if q.dim() != 4 or q.shape != k.shape:
+        raise ValueError("q and k must both be [B, L, heads, head_dim]")
+    B, L, Hh, D = q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != L:
+        raise ValueError("grid does not match the sequence length")
+    d_t, d_h, d_w = default_split(D) if split is None else split
+    if inplace:
+        q_out, k_out = q, k
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    w_ptrs = []
+    for w, name in ((wq, "wq"), (wk, "wk")):
+        if w is None:
+            w_ptrs.append(None)
+        else:
+            if tuple(w.shape) != (norm_group,):
+                raise ValueError(f"{name} must have norm_group entries")
+            w_ptrs.append(_dev(w, name, torch.float32))
+    _check("vdit_qk_norm_rope_3d", lib().vdit_qk_norm_rope_3d(
+        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
+        _dev(k_out, "k_out", torch.bfloat16), w_ptrs[0], w_ptrs[1], int(norm_group), float(eps),
+        B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
     return q_out, k_out
 
 

@@ -292,4 +292,175 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat1
   }
 }
 
+// ---------------------------------------------------------------------------
+// Q/K RMSNorm fused with the 3D RoPE
+// ---------------------------------------------------------------------------
+//
+// "How AI Generates Video: Inside Sora and Wan2.1 on a Real GPU", section 5
+// (Sub-Layer 1): the projected Q and K are RMS-normalised, then rotated.  One
+// HBM pass does both.  A CTA walks its tokens (blockIdx.x + k * gridDim.x);
+// thread 0 streams each token's Q and K rows (heads*D bf16 each) into a ring
+// of kNormStages shared-memory stages with bulk copies, kNormStages tokens
+// ahead, so that several tokens per CTA are in flight.  For the token at hand
+// threads 0..127 take Q and 128..255 K, thread t the 16-byte vectors t,
+// t + 128, ...; each group of `group` channels is summed in float32 (a
+// segmented shuffle reduction when a group's vectors sit in consecutive lanes of
+// one warp, or warp sums added over the tensor's four warps when the group is
+// the whole token); then y = x * rsqrt(mean + eps) * weight[channel mod group],
+// rotated like rope3d_kernel (separately rounded float32 products), rounded
+// once to bfloat16 and stored.  A CTA-wide barrier at the end of each token
+// frees its stage for the copy kNormStages tokens later.  The (cos, sin) of
+// every pair at every position of its axis (Tg x d_t/2 + Hg x d_h/2 + Wg x
+// d_w/2 entries) are built once per CTA in shared memory, after the ring, so
+// that a token's rotation is a table lookup.
+
+constexpr int kNormThreads = 256;
+constexpr int kNormStages = 4;
+constexpr int kNormVecs = 8;        // vectors per thread: heads * head_dim <= 128 * 8 * 8 = 8,192
+constexpr int kSiteNormFull = 30, kSiteNormDrain = 31;   // watchdog wait sites
+constexpr int kNormMaxTable = 8192;  // (cos, sin) table entries: Tg*d_t/2 + Hg*d_h/2 + Wg*d_w/2
+
+template <bool kWide>   // the group is the token's whole heads*D vector
+__global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
+    const __nv_bfloat16* q_in, const __nv_bfloat16* k_in, __nv_bfloat16* q_out, __nv_bfloat16* k_out,
+    const float* __restrict__ wq, const float* __restrict__ wk, RopeShape s, int group, float eps, double theta) {
+  __shared__ float wsum[2][4];                          // [tensor][warp]: sums of squares
+  __shared__ float2 cs[2][kRopeMaxPairs];              // the token's pairs, by token parity
+  __shared__ __align__(8) uint64_t full[kNormStages];
+  if (__syncthreads_or(watchdog_tripped())) return;    // all threads of the CTA decide alike
+
+  const int vec_per_head = s.D / 8;
+  const int nv = s.heads * vec_per_head;                // vectors per token and tensor
+  uint4* ring = reinterpret_cast<uint4*>(dyn_smem);    // [stage][Q row, K row] of nv vectors each
+  // per-axis tables: time [Tg][d_t/2], then height [Hg][d_h/2], then width [Wg][d_w/2]
+  float2* tab = reinterpret_cast<float2*>(ring + (size_t)kNormStages * 2 * nv);
+  const int pt = s.d_t / 2, ph = s.d_h / 2, pw = s.d_w / 2;
+  const int Tg = (int)(s.L / ((long long)s.Hg * s.Wg));
+  const int off_h = Tg * pt, off_w = off_h + s.Hg * ph, n_tab = off_w + s.Wg * pw;
+  for (int x = threadIdx.x; x < n_tab; x += blockDim.x) {
+    int pos, i, d;
+    if (x < off_h) { pos = x / pt; i = x - pos * pt; d = s.d_t; }
+    else if (x < off_w) { pos = (x - off_h) / ph; i = x - off_h - pos * ph; d = s.d_h; }
+    else { pos = (x - off_w) / pw; i = x - off_w - pos * pw; d = s.d_w; }
+    double sn, cn;
+    sincos((double)pos * (1.0 / pow(theta, (double)(2 * i) / (double)d)), &sn, &cn);
+    tab[x] = make_float2((float)cn, (float)sn);
+  }
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kNormStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const uint32_t row_bytes = (uint32_t)nv * 16u;
+  const long long n_my = (s.ntok - 1 - blockIdx.x) / gridDim.x + 1;   // grid <= ntok
+  auto issue = [&](long long k) {                       // thread 0: token k of this CTA into its stage
+    const int st = (int)(k % kNormStages);
+    const long long tok = blockIdx.x + k * gridDim.x;
+    mbar_arrive_expect_tx(&full[st], 2u * row_bytes);
+    bulk_load(ring + (size_t)st * 2 * nv, q_in + tok * nv * 8, row_bytes, &full[st]);
+    bulk_load(ring + (size_t)st * 2 * nv + nv, k_in + tok * nv * 8, row_bytes, &full[st]);
+  };
+  long long issued = n_my < kNormStages ? n_my : kNormStages;
+  if (threadIdx.x == 0)
+    for (long long k = 0; k < issued; ++k) issue(k);
+
+  const int which = threadIdx.x >> 7;                   // 0: Q, 1: K
+  const int t = threadIdx.x & 127;
+  const int lane = threadIdx.x & 31, wt = t >> 5;       // warp within the tensor's four
+  const int gv = group / 8;                             // vectors per group
+  const float inv_group = 1.f / (float)group;
+  const float* w = which ? wk : wq;
+  long long k = 0;
+  for (; k < n_my; ++k) {
+    const long long tok = blockIdx.x + k * gridDim.x;
+    const int l = (int)(tok % s.L);
+    const int par = (int)(k & 1);
+    if (threadIdx.x < (unsigned)(pt + ph + pw)) {       // the token's row of pairs, from the axis tables
+      const int pp = threadIdx.x;
+      float2 c;
+      if (pp < pt) c = tab[(l / (s.Hg * s.Wg)) * pt + pp];
+      else if (pp < pt + ph) c = tab[off_h + ((l / s.Wg) % s.Hg) * ph + (pp - pt)];
+      else c = tab[off_w + (l % s.Wg) * pw + (pp - pt - ph)];
+      cs[par][pp] = c;
+    }
+    const int st = (int)(k % kNormStages);
+    const bool okw = mbar_wait(&full[st], (uint32_t)((k / kNormStages) & 1), kSiteNormFull);
+    if (!__syncthreads_and(okw)) break;                 // also publishes cs[par]
+    const uint4* sv = ring + (size_t)st * 2 * nv + (size_t)which * nv;
+    uint4 v[kNormVecs];
+#pragma unroll
+    for (int r = 0; r < kNormVecs; ++r) {
+      const int e = t + 128 * r;
+      v[r] = e < nv ? sv[e] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    auto vec_sq = [&](const uint4& x) -> float {
+      const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+      float a = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&u[m]);
+        const float x0 = __low2float(pr), x1 = __high2float(pr);
+        a = fmaf(x0, x0, a);
+        a = fmaf(x1, x1, a);
+      }
+      return a;
+    };
+    float tok_sq = 0.f;
+    if (kWide) {
+#pragma unroll
+      for (int r = 0; r < kNormVecs; ++r) tok_sq += vec_sq(v[r]);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) tok_sq += __shfl_xor_sync(0xffffffffu, tok_sq, o);
+      if (lane == 0) wsum[which][wt] = tok_sq;
+      __syncthreads();
+      tok_sq = (wsum[which][0] + wsum[which][1]) + (wsum[which][2] + wsum[which][3]);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(which ? k_out : q_out) + tok * nv;
+#pragma unroll
+    for (int r = 0; r < kNormVecs; ++r) {
+      float sq = tok_sq;
+      if (!kWide) {                                     // the group's gv vectors: gv consecutive lanes
+        sq = vec_sq(v[r]);
+        for (int o = gv >> 1; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      const int e = t + 128 * r;
+      if (e < nv) {
+        const float scale = rsqrtf(fmaf(sq, inv_group, eps));
+        const int c0 = (e * 8) % group;                 // channel of the vector's first element in its group
+        float wv[8];
+        if (w != nullptr) {
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + c0));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + c0 + 4));
+          wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+          wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) wv[m] = 1.f;
+        }
+        const int p0 = (e % vec_per_head) * 4;
+        uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&u[m]);
+          const float x0 = __fmul_rn(__fmul_rn(__low2float(pr), scale), wv[2 * m]);
+          const float x1 = __fmul_rn(__fmul_rn(__high2float(pr), scale), wv[2 * m + 1]);
+          const float2 c = cs[par][p0 + m];
+          const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
+          const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
+          u[m] = pack_bf16x2(re, im);
+        }
+        dst[e] = make_uint4(u[0], u[1], u[2], u[3]);
+      }
+    }
+    __syncthreads();                                    // the stage (and wsum) is free
+    if (threadIdx.x == 0 && issued < n_my) issue(issued++);
+  }
+  // No copy may still be landing in shared memory when the CTA exits (only
+  // when a wait above ran out can tokens k .. issued-1 still be in flight).
+  if (threadIdx.x == 0)
+    for (long long k2 = k; k2 < issued; ++k2)
+      mbar_drain_site(&full[k2 % kNormStages], (uint32_t)((k2 / kNormStages) & 1), kSiteNormDrain);
+}
+
 }  // namespace vdit

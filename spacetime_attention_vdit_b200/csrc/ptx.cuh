@@ -111,6 +111,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
   }
 }
 
+// A wait bounded by time only, for draining copies before a CTA exits; a wait
+// that runs out is recorded at `site`.
+__device__ __forceinline__ void mbar_drain_site(uint64_t* bar, uint32_t parity, int site) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) { watchdog_trip(site); return; }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Proxy fences
 // ---------------------------------------------------------------------------
@@ -122,6 +131,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
+// Untiled bulk copy global -> shared (no multicast): `bytes` and both
+// addresses 16-byte aligned; completion is counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // TMA (cp.async.bulk.tensor), tiled mode, no multicast
 // ---------------------------------------------------------------------------
 

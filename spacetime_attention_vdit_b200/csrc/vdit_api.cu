@@ -323,6 +323,59 @@ int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, i
   return last_launch_status();
 }
 
+int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* wq,
+                         const float* wk, int norm_group, float eps, int B, int Tg, int Hg, int Wg, int heads,
+                         int head_dim, int d_t, int d_h, int d_w, float theta, vdit_stream_t stream) {
+  if (!q_in || !k_in || !q_out || !k_out) return VDIT_ERR_NULL;
+  if (B <= 0 || Tg <= 0 || Hg <= 0 || Wg <= 0 || heads <= 0 || head_dim <= 0) return VDIT_ERR_SHAPE;
+  if (d_t < 0 || d_h < 0 || d_w < 0 || (d_t | d_h | d_w) & 1 || d_t + d_h + d_w != head_dim) return VDIT_ERR_SHAPE;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return VDIT_ERR_SHAPE;
+  const long long width = (long long)heads * head_dim;
+  if (norm_group <= 0 || width % norm_group != 0 || !(eps >= 0.f) || !std::isfinite(eps)) return VDIT_ERR_SHAPE;
+  if (head_dim % 8 != 0 || head_dim / 2 > kRopeMaxPairs || norm_group % 8 != 0) return VDIT_ERR_UNSUPPORTED;
+  const int gv = norm_group / 8;                       // 16-byte vectors per group
+  const bool wide = norm_group == width;               // one group: the token's whole vector
+  if (!wide && 32 % gv != 0) return VDIT_ERR_UNSUPPORTED;
+  if (width > 128LL * 8 * kNormVecs) return VDIT_ERR_UNSUPPORTED;
+  if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
+      (wq && !aligned16(wq)) || (wk && !aligned16(wk)))
+    return VDIT_ERR_ALIGN;
+  const long long L = (long long)Tg * Hg * Wg;
+  if (L > 0x7fffffffLL || (double)B * (double)L * (double)width > 4.0e18) return VDIT_ERR_SHAPE;
+  RopeShape s;
+  s.ntok = (long long)B * L;
+  s.L = (int)L; s.Hg = Hg; s.Wg = Wg;
+  s.heads = heads; s.D = head_dim;
+  s.pt_end = d_t / 2; s.ph_end = (d_t + d_h) / 2;
+  s.d_t = d_t; s.d_h = d_h; s.d_w = d_w;
+  const long long cap = (long long)sm_count() * 2;
+  const unsigned grid = (unsigned)(s.ntok < cap ? s.ntok : cap);
+  // the ring (Q and K rows of kNormStages tokens) and the per-axis (cos, sin) tables
+  const long long tab = (long long)Tg * (d_t / 2) + (long long)Hg * (d_h / 2) + (long long)Wg * (d_w / 2);
+  if (tab > kNormMaxTable) return VDIT_ERR_UNSUPPORTED;
+  const int smem = kNormStages * 2 * (int)width * 2 + (int)tab * 8;
+  {
+    static bool done_n[kMaxDevices] = {}, done_w[kMaxDevices] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ensure_smem(qk_norm_rope3d_kernel<false>, kNormStages * 2 * 8192 * 2 + kNormMaxTable * 8, done_n) ||
+        !ensure_smem(qk_norm_rope3d_kernel<true>, kNormStages * 2 * 8192 * 2 + kNormMaxTable * 8, done_w))
+      return VDIT_ERR_CUDA;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* qi = static_cast<const __nv_bfloat16*>(q_in);
+  const auto* ki = static_cast<const __nv_bfloat16*>(k_in);
+  auto* qo = static_cast<__nv_bfloat16*>(q_out);
+  auto* ko = static_cast<__nv_bfloat16*>(k_out);
+  if (wide)
+    qk_norm_rope3d_kernel<true><<<grid, kNormThreads, smem, st>>>(qi, ki, qo, ko, wq, wk, s, norm_group, eps,
+                                                               (double)theta);
+  else
+    qk_norm_rope3d_kernel<false><<<grid, kNormThreads, smem, st>>>(qi, ki, qo, ko, wq, wk, s, norm_group, eps,
+                                                                (double)theta);
+  return last_launch_status();
+}
+
 int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* lse, int B, int L, int heads,
                    int head_dim, float scale, vdit_stream_t stream) {
   const int rc = check_attn_args(q, k, v, o, lse, B, L, heads, head_dim);

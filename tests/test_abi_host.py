@@ -77,6 +77,25 @@ def test_rope_validation(L):
     assert rope(L, ko=MIS) == ALIGN
 
 
+def norm_rope(L, q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, wq=None, wk=None, group=128, eps=1e-6, B=1, Tg=2, Hg=3,
+              Wg=4, heads=2, D=128, split=(44, 42, 42), theta=10000.0):
+    return L.vdit_qk_norm_rope_3d(q, k, qo, ko, wq, wk, group, ctypes.c_float(eps), B, Tg, Hg, Wg, heads, D,
+                                  *split, ctypes.c_float(theta), None)
+
+
+def test_qk_norm_rope_validation(L):
+    assert norm_rope(L, q=None) == NULL
+    assert norm_rope(L, group=0) == SHAPE
+    assert norm_rope(L, group=96) == SHAPE            # does not divide heads * head_dim = 256
+    assert norm_rope(L, eps=-1.0) == SHAPE
+    assert norm_rope(L, split=(44, 42, 40)) == SHAPE
+    assert norm_rope(L, group=12, D=24, split=(8, 8, 8)) == UNSUP        # not a multiple of 8
+    assert norm_rope(L, heads=3, D=32, split=(12, 10, 10), group=48) == UNSUP   # 6 vectors, not the token
+    assert norm_rope(L, heads=72, D=128) == UNSUP   # 9,216 channels per token
+    assert norm_rope(L, wq=MIS) == ALIGN
+    assert norm_rope(L, ko=MIS) == ALIGN
+
+
 def attn(L, fn="vdit_attn_full", q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, dims=(1, 256, 2, 128)):
     f = getattr(L, fn)
     return f(q, k, v, o, lse, *dims, ctypes.c_float(0.0), None)
@@ -143,7 +162,7 @@ def test_register_budget_fits_each_sm_subpartition():
         if m and name:
             regs[name] = int(m.group(1))
     threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256,
-               "patchify122_f32_kernel": 128}
+               "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256}
 
     def block_of(kname):
         for key, t in threads.items():
