@@ -23,8 +23,8 @@ import os
 
 import torch
 
-__all__ = ["VditError", "lib", "patchify_3d", "rope_3d", "attn_full", "attn_divided_time",
-           "attn_divided_space", "device_status", "status_string", "default_split", "LIB_PATH"]
+__all__ = ["VditError", "lib", "patchify_3d", "rope_3d", "qk_norm_rope_3d", "attn_full", "attn_divided_time",
+           "attn_divided_space", "attn_cross", "device_status", "status_string", "default_split", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
 
