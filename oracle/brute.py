@@ -68,3 +68,24 @@ def rms_norm(x, weight, eps):
     ms = sum(a * a for a in x) / len(x)
     r = math.sqrt(ms + eps)
     return [a / r * w for a, w in zip(x, weight)]
+
+
+def unpatchify(tokens, C, grid, pt, ph, pw):
+    """latent[n][c][t'*pt + dt][h'*ph + dh][w'*pw + dw]
+    = tokens[n][(t'*H' + h')*W' + w'][((c*pt + dt)*ph + dh)*pw + dw], as nested lists."""
+    Tg, Hg, Wg = grid
+    N = len(tokens)
+    out = [[[[[0.0] * (Wg * pw) for _ in range(Hg * ph)] for _ in range(Tg * pt)] for _ in range(C)]
+           for _ in range(N)]
+    for n in range(N):
+        for tq in range(Tg):
+            for hq in range(Hg):
+                for wq in range(Wg):
+                    row = (tq * Hg + hq) * Wg + wq
+                    for c in range(C):
+                        for dt in range(pt):
+                            for dh in range(ph):
+                                for dw in range(pw):
+                                    col = ((c * pt + dt) * ph + dh) * pw + dw
+                                    out[n][c][tq * pt + dt][hq * ph + dh][wq * pw + dw] = tokens[n][row][col]
+    return out

@@ -67,6 +67,35 @@ def patchify(latent: np.ndarray, pt: int, ph: int, pw: int) -> np.ndarray:
     return np.ascontiguousarray(x.reshape(N, Tg * Hg * Wg, C * pt * ph * pw))
 
 
+def unpatchify(tokens: np.ndarray, C: int, grid, pt: int, ph: int, pw: int) -> np.ndarray:
+    """Put every token's brick back: ``[N, Tg*Hg*Wg, C*pt*ph*pw]`` ->
+    ``[N, C, Tg*pt, Hg*ph, Wg*pw]``, the inverse of ``patchify`` (the last step
+    of the transformer maps its tokens back to the latent clip the same way the
+    first cut it; same feature order)."""
+    N, L, F = tokens.shape
+    Tg, Hg, Wg = grid
+    if L != Tg * Hg * Wg or F != C * pt * ph * pw:
+        raise ValueError("tokens do not match the grid and brick")
+    x = tokens.reshape(N, Tg, Hg, Wg, C, pt, ph, pw)
+    # -> N, C, Tg, pt, Hg, ph, Wg, pw
+    x = x.transpose(0, 4, 1, 5, 2, 6, 3, 7)
+    return np.ascontiguousarray(x.reshape(N, C, Tg * pt, Hg * ph, Wg * pw))
+
+
+def patch_embed(latent: np.ndarray, weight: np.ndarray, bias, pt: int, ph: int, pw: int) -> np.ndarray:
+    """The patch embedding: a Conv3d whose stride equals its kernel (cheatsheet
+    "Tiny video DiT"; towardsai section 4: each 1x2x2 brick of 16 latent channels
+    becomes one model-width token), i.e. patchify then a matrix product, in
+    float64.  ``weight`` is the Conv3d weight [dim, C, pt, ph, pw] flattened to
+    [dim, C*pt*ph*pw]; ``bias`` is [dim] or None.  Returns [N, L, dim]."""
+    tok = patchify(np.asarray(latent, dtype=np.float64), pt, ph, pw)
+    w = np.asarray(weight, dtype=np.float64)
+    y = tok @ w.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)
+    return y
+
+
 # ----------------------------------------------------------------------------
 # 3D rotary position embedding
 # ----------------------------------------------------------------------------

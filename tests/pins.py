@@ -176,6 +176,81 @@ ROPE_PINS = [pin_rope_onehot, pin_rope_complex, pin_rope_relative, pin_rope_norm
              pin_rope_brute]
 
 # ----------------------------------------------------------------------------
+# Patch embedding and unpatchify  (cheatsheet "Tiny video DiT": a Conv3d whose
+# stride equals its kernel; towardsai section 4: bricks to model-width tokens)
+# ----------------------------------------------------------------------------
+
+
+def _onehot_brick_weight(C, pt, ph, pw):
+    """Conv weight [F, C, pt, ph, pw] with weight[f, c, dt, dh, dw] = 1 iff f is the
+    brick feature index of (c, dt, dh, dw)."""
+    F = C * pt * ph * pw
+    w = np.zeros((F, C, pt, ph, pw))
+    for c in range(C):
+        for dt in range(pt):
+            for dh in range(ph):
+                for dw in range(pw):
+                    w[((c * pt + dt) * ph + dh) * pw + dw, c, dt, dh, dw] = 1.0
+    return w
+
+
+def pin_embed_conv3d(patch_embed):
+    """torch's conv3d in float64, stride = kernel, then channels-last tokens."""
+    g = np.random.default_rng(51)
+    for (N, C, T, H, W), (pt, ph, pw), dim in (((2, 4, 3, 6, 8), (1, 2, 2), 24), ((1, 2, 4, 5, 7), (2, 2, 3), 10)):
+        x = g.standard_normal((N, C, T, H, W))
+        w = g.standard_normal((dim, C * pt * ph * pw))
+        b = g.standard_normal(dim)
+        got = patch_embed(x, w, b, pt, ph, pw)
+        y = torch.nn.functional.conv3d(torch.from_numpy(x), torch.from_numpy(w.reshape(dim, C, pt, ph, pw)),
+                                       torch.from_numpy(b), stride=(pt, ph, pw)).numpy()
+        exp = y.reshape(N, dim, -1).transpose(0, 2, 1)
+        assert np.allclose(got, exp, atol=1e-12)
+
+
+def pin_embed_identity_and_brute(patch_embed):
+    """The one-hot weight turns the embedding into patchify itself; scalar loops
+    agree on a tiny clip with a bias."""
+    g = np.random.default_rng(52)
+    x = g.standard_normal((1, 3, 2, 4, 4))
+    F = 3 * 1 * 2 * 2
+    eye = np.eye(F)
+    assert np.array_equal(patch_embed(x, eye, None, 1, 2, 2), brute_tokens(x, 1, 2, 2))
+    w = g.standard_normal((5, F))
+    b = g.standard_normal(5)
+    got = patch_embed(x, w, b, 1, 2, 2)
+    tok = brute.patchify(x.tolist(), 1, 2, 2)
+    for l in range(len(tok[0])):
+        for o in range(5):
+            assert abs(got[0, l, o] - (sum(tok[0][l][f] * w[o, f] for f in range(F)) + b[o])) < 1e-12
+
+
+def brute_tokens(x, pt, ph, pw):
+    return np.array(brute.patchify(x.tolist(), pt, ph, pw))
+
+
+def pin_unpatchify(unpatchify):
+    """The inverse of patchify (exactly), torch's conv_transpose3d with the one-hot
+    brick weight in float64, and scalar loops."""
+    g = np.random.default_rng(53)
+    for (N, C, T, H, W), (pt, ph, pw) in (((2, 3, 4, 6, 8), (1, 2, 2)), ((1, 2, 4, 6, 6), (2, 3, 2))):
+        x = g.standard_normal((N, C, T, H, W))
+        grid = (T // pt, H // ph, W // pw)
+        tok = brute_tokens(x, pt, ph, pw)
+        assert np.array_equal(unpatchify(tok, C, grid, pt, ph, pw), x)
+        y = torch.nn.functional.conv_transpose3d(
+            torch.from_numpy(tok.transpose(0, 2, 1).reshape(N, -1, *grid)),
+            torch.from_numpy(_onehot_brick_weight(C, pt, ph, pw)), stride=(pt, ph, pw)).numpy()
+        assert np.allclose(unpatchify(tok, C, grid, pt, ph, pw), y, atol=0)
+    tok = g.standard_normal((1, 2 * 2 * 3, 8))
+    assert np.array_equal(unpatchify(tok, 2, (2, 2, 3), 1, 2, 2),
+                          np.array(brute.unpatchify(tok.tolist(), 2, (2, 2, 3), 1, 2, 2)))
+
+
+EMBED_PINS = [pin_embed_conv3d, pin_embed_identity_and_brute]
+UNPATCHIFY_PINS = [pin_unpatchify]
+
+# ----------------------------------------------------------------------------
 # Q/K RMSNorm before the 3D RoPE  (towardsai section 5, Sub-Layer 1)
 # ----------------------------------------------------------------------------
 

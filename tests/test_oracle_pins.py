@@ -32,6 +32,16 @@ def test_norm_pins(pin):
     pin(ref.qk_norm_rope_3d)
 
 
+@pytest.mark.parametrize("pin", pins.EMBED_PINS, ids=lambda p: p.__name__)
+def test_embed_pins(pin):
+    pin(ref.patch_embed)
+
+
+def test_unpatchify_pins():
+    for pin in pins.UNPATCHIFY_PINS:
+        pin(ref.unpatchify)
+
+
 def test_divided_pins():
     pins.pin_divided_time(ref.divided_time)
     pins.pin_divided_space(ref.divided_space)
@@ -195,3 +205,32 @@ def test_norm_mistakes_caught(kw):
         pin(_norm_variant)
     bad = lambda *a, **k: _norm_variant(*a, **k, **kw)
     assert _fails(pins.NORM_PINS, bad) >= 1
+
+
+# ---- patch embedding and unpatchify: planted mistakes
+
+
+def embed_feature_order_swapped(latent, weight, bias, pt, ph, pw):
+    """Mistake: brick features (dt, dh, dw, c) against a (c, dt, dh, dw) weight."""
+    return patchify_feature_order_swapped(latent, pt, ph, pw) @ np.asarray(weight).T + (0 if bias is None else bias)
+
+
+def embed_bias_dropped(latent, weight, bias, pt, ph, pw):
+    return ref.patch_embed(latent, weight, None, pt, ph, pw)
+
+
+def unpatchify_spatial_swapped(tokens, C, grid, pt, ph, pw):
+    """Mistake: brick rows and columns exchanged on the way back."""
+    N = tokens.shape[0]
+    Tg, Hg, Wg = grid
+    x = tokens.reshape(N, Tg, Hg, Wg, C, pt, ph, pw).transpose(0, 4, 1, 5, 2, 7, 3, 6)
+    return np.ascontiguousarray(x.reshape(N, C, Tg * pt, Hg * pw, Wg * ph))
+
+
+@pytest.mark.parametrize("bad", [embed_feature_order_swapped, embed_bias_dropped], ids=lambda f: f.__name__)
+def test_embed_mistakes_caught(bad):
+    assert _fails(pins.EMBED_PINS, bad) >= 1
+
+
+def test_unpatchify_mistake_caught():
+    assert _fails(pins.UNPATCHIFY_PINS, unpatchify_spatial_swapped) == 1
