@@ -530,6 +530,41 @@ def main():
         cross["qk_norm_rope"] = {"norm_group": width, "ms": nms, "gb_s": nbytes / (nms * 1e-3) / 1e9,
                                  "frac_hbm": nbytes / (nms * 1e-3) / 1e9 / peaks["hbm_gbs"], "bytes": nbytes}
         del qn, kn
+        # next row: the patch embedding (patchify and the Conv3d weight on the tensor
+        # cores) to the model width heads*D of this workload
+        dim = Hh * D
+        wemb = (torch.randn(dim, LATENT_C * PATCH[0] * PATCH[1] * PATCH[2], device=dev) / 8).to(torch.bfloat16)
+        bemb = torch.randn(dim, device=dev)
+        emb = torch.empty((d["B"], L, dim), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            vd.patch_embed_3d(lat, wemb, PATCH, bemb, out=emb)
+        a.record(stream)
+        for _ in range(reps):
+            vd.patch_embed_3d(lat, wemb, PATCH, bemb, out=emb)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = a.elapsed_time(b_) / reps
+        ebytes = lat.numel() * 4 + wemb.numel() * 2 + dim * 4 + emb.numel() * 2
+        cross["patch_embed"] = {"dim": dim, "ms": ems, "gb_s": ebytes / (ems * 1e-3) / 1e9,
+                                "frac_hbm": ebytes / (ems * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "tflops": 2.0 * emb.numel() * wemb.shape[1] / (ems * 1e-3) / 1e12, "bytes": ebytes}
+        del wemb, bemb, emb
+        # next row: unpatchify, measured where bandwidth shows (64 clips at 720p)
+        big_tok = torch.empty((64, 21 * 45 * 80, LATENT_C * 4), dtype=torch.float32, device=dev).normal_()
+        big = torch.empty((64, LATENT_C, 21, 90, 160), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            vd.unpatchify_3d(big_tok, LATENT_C, (21, 45, 80), PATCH, out=big)
+        a.record(stream)
+        for _ in range(5):
+            vd.unpatchify_3d(big_tok, LATENT_C, (21, 45, 80), PATCH, out=big)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        ums = a.elapsed_time(b_) / 5
+        ubytes = 2 * big.numel() * 4
+        cross["unpatchify_64_clips_720p"] = {"ms": ums, "gb_s": ubytes / (ums * 1e-3) / 1e9,
+                                             "frac_hbm": ubytes / (ums * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                             "bytes": ubytes}
+        del big_tok, big
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -7,6 +7,8 @@
  *
  *   latent clip [N, C, T, H, W]
  *     -> vdit_patchify_3d        cut into (pt, ph, pw) spacetime bricks, one token each
+ *        (or vdit_patch_embed_3d: patchify and the Conv3d weight in one pass,
+ *         tokens of the model width)
  *     -> (projection to per-head Q, K, V: done by the caller)
  *     -> vdit_rope_3d            factorised 3D rotary positions on Q and K
  *        (or vdit_qk_norm_rope_3d: RMSNorm of Q and K, then the same rotation)
@@ -16,6 +18,7 @@
  *        vdit_attn_divided_space attention over the H'*W' tokens of each frame
  *     -> vdit_attn_cross         the video tokens attend to the text tokens' keys
  *                                and values (the block's second attention)
+ *   and at the end: vdit_unpatchify_3d, tokens back to the latent clip
  *
  * Sources (page title, section):
  *   [towardsai]  "How AI Generates Video: Inside Sora and Wan2.1 on a Real GPU",
@@ -128,6 +131,38 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
 int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
                  int B, int Tg, int Hg, int Wg, int heads, int head_dim,
                  int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
+
+/*
+ * vdit_patch_embed_3d - the patch embedding: a Conv3d whose stride equals its
+ * kernel [cheatsheet "Tiny video DiT"; towardsai s.4: each 1x2x2 brick of the
+ * 16-channel latent becomes one token of the model width], on the tensor cores.
+ *
+ *   out[n, l, o] = sum_f brick(n, l)[f] * weight[o, f] + bias[o]
+ *
+ * with brick(n, l) the token's C*pt*ph*pw latent values in vdit_patchify_3d's
+ * feature order.  latent: float32 [N, C, T, H, W] (rounded to bfloat16, nearest
+ * even, as the tensor-core operand); weight: bfloat16 [dim, C*pt*ph*pw] (the
+ * Conv3d weight [dim, C, pt, ph, pw] flattened), 16-byte aligned; bias: NULL
+ * or float32 [dim], 16-byte aligned; out: bfloat16 [N, Tg*Hg*Wg, dim], float32
+ * accumulation, rounded once.  Extents that do not divide are floored.
+ * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED
+ * (C*pt*ph*pw other than 64, or dim not a multiple of 256), VDIT_ERR_CUDA.
+ */
+int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bias, void* out,
+                        int N, int C, int T, int H, int W, int pt, int ph, int pw, int dim,
+                        vdit_stream_t stream);
+
+/*
+ * vdit_unpatchify_3d - the inverse of vdit_patchify_3d: every token's brick is
+ * put back, tokens [N, Tg*Hg*Wg, C*pt*ph*pw] -> latent [N, C, Tg*pt, Hg*ph,
+ * Wg*pw] (the map from the transformer's last output to the latent clip).  A
+ * permutation of values: bit exact, dtype VDIT_F32 or VDIT_BF16.  The buffers
+ * must not overlap.
+ * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_UNSUPPORTED (dtype, or a token
+ * wider than 32 KB), VDIT_ERR_CUDA.
+ */
+int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C, int Tg, int Hg, int Wg,
+                       int pt, int ph, int pw, vdit_stream_t stream);
 
 /*
  * vdit_qk_norm_rope_3d - RMSNorm of Q and K, then the 3D RoPE, in one pass

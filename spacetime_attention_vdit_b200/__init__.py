@@ -23,7 +23,7 @@ import os
 
 import torch
 
-__all__ = ["VditError", "lib", "patchify_3d", "rope_3d", "qk_norm_rope_3d", "attn_full", "attn_divided_time",
+__all__ = ["VditError", "lib", "patchify_3d", "patch_embed_3d", "unpatchify_3d", "rope_3d", "qk_norm_rope_3d", "attn_full", "attn_divided_time",
            "attn_divided_space", "attn_cross", "device_status", "status_string", "default_split", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
@@ -48,6 +48,8 @@ _SIGNATURES = {
     "vdit_patchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_rope_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_full": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P],
+    "vdit_patch_embed_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
+    "vdit_unpatchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_qk_norm_rope_3d": [_P, _P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_time": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_divided_space": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
@@ -153,6 +155,53 @@ def rope_3d(q: torch.Tensor, k: torch.Tensor, grid, split=None, theta: float = 1
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
         _dev(k_out, "k_out", torch.bfloat16), B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
     return q_out, k_out
+
+
+def patch_embed_3d(latent: torch.Tensor, weight: torch.Tensor, patch=(1, 2, 2), bias=None, out=None,
+                   stream=None):
+    """The Conv3d patch embedding on the tensor cores: latent float32 [N, C, T, H, W],
+    weight bfloat16 [dim, C*pt*ph*pw] (or the Conv3d's [dim, C, pt, ph, pw]),
+    bias float32 [dim] or None -> bfloat16 [N, L, dim]."""
+    if latent.dim() != 5:
+        raise ValueError("latent must be [N, C, T, H, W]")
+    N, C, T, H, W = latent.shape
+    pt, ph, pw = patch
+    w = weight.reshape(weight.shape[0], -1)
+    dim = w.shape[0]
+    L = (T // pt) * (H // ph) * (W // pw)
+    if out is None:
+        out = torch.empty((N, L, dim), dtype=torch.bfloat16, device=latent.device)
+    elif tuple(out.shape) != (N, L, dim):
+        raise ValueError(f"out must be {(N, L, dim)}")
+    _check("vdit_patch_embed_3d", lib().vdit_patch_embed_3d(
+        _dev(latent, "latent", torch.float32), _dev(w, "weight", torch.bfloat16),
+        None if bias is None else _dev(bias, "bias", torch.float32), _dev(out, "out", torch.bfloat16),
+        N, C, T, H, W, pt, ph, pw, dim, _stream(stream)))
+    return out
+
+
+def unpatchify_3d(tokens: torch.Tensor, C: int, grid, patch=(1, 2, 2), out=None, stream=None):
+    """Tokens [N, Tg*Hg*Wg, C*pt*ph*pw] (float32 or bfloat16) back to the latent
+    [N, C, Tg*pt, Hg*ph, Wg*pw]: the inverse of :func:`patchify_3d`."""
+    if tokens.dim() != 3:
+        raise ValueError("tokens must be [N, L, features]")
+    N, L, F = tokens.shape
+    Tg, Hg, Wg = grid
+    pt, ph, pw = patch
+    if L != Tg * Hg * Wg or F != C * pt * ph * pw:
+        raise ValueError("tokens do not match the grid and the brick")
+    dt = {torch.float32: 0, torch.bfloat16: 1}.get(tokens.dtype)
+    if dt is None:
+        raise ValueError("tokens must be float32 or bfloat16")
+    shape = (N, C, Tg * pt, Hg * ph, Wg * pw)
+    if out is None:
+        out = torch.empty(shape, dtype=tokens.dtype, device=tokens.device)
+    elif tuple(out.shape) != shape:
+        raise ValueError(f"out must be {shape}")
+    _check("vdit_unpatchify_3d", lib().vdit_unpatchify_3d(
+        _dev(tokens, "tokens", tokens.dtype), _dev(out, "out", tokens.dtype), dt, N, C, Tg, Hg, Wg, pt, ph, pw,
+        _stream(stream)))
+    return out
 
 
 def qk_norm_rope_3d(q: torch.Tensor, k: torch.Tensor, grid, norm_group: int, wq=None, wk=None,

@@ -101,13 +101,6 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// All 32 lanes wait; the result is made warp-uniform, so that a lane whose
-// wait ran out never leaves its warp-mates inside a .sync.aligned instruction.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int site) {
-  const bool ok = mbar_wait(bar, parity, site);
-  return __all_sync(0xffffffffu, ok) != 0;
-}
-
 // 2^x on the FMA pipe, for x <= 8: x = n + f with n = rint(x) (the 1.5 * 2^23
 // rounding constant) and |f| <= 1/2; 2^f from a cubic fitted here by
 // relative-error least squares on [-1/2, 1/2] (max relative error 7.8e-5, below

@@ -15,6 +15,7 @@
 #include "attn_tcgen05.cuh"
 #include "attn_time_short.cuh"
 #include "patchify_rope.cuh"
+#include "patch_embed.cuh"
 
 namespace {
 
@@ -88,6 +89,20 @@ bool make_qkv_map(CUtensorMap* map, const void* base, int D, int heads, long lon
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D view {cols, rows} of a row-major bf16 matrix (cols a multiple of 8);
+// box {box_cols, box_rows}, 128-byte swizzle when a box row is 128 bytes.
+bool make_2d_map(CUtensorMap* map, const void* base, long long cols, long long rows, int box_cols, int box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---------------------------------------------------------------------------
@@ -295,6 +310,71 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype, int N, int C, 
   else
     patchify3d_kernel<__nv_bfloat16><<<grid, kPatchifyThreads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(latent), static_cast<__nv_bfloat16*>(tokens), s);
+  return last_launch_status();
+}
+
+int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C, int Tg, int Hg, int Wg, int pt,
+                       int ph, int pw, vdit_stream_t stream) {
+  if (!tokens || !latent) return VDIT_ERR_NULL;
+  if (dtype != VDIT_F32 && dtype != VDIT_BF16) return VDIT_ERR_UNSUPPORTED;
+  if (N <= 0 || C <= 0 || Tg <= 0 || Hg <= 0 || Wg <= 0 || pt <= 0 || ph <= 0 || pw <= 0) return VDIT_ERR_SHAPE;
+  const long long F = (long long)C * pt * ph * pw;
+  const long long ntok = (long long)N * Tg * Hg * Wg;
+  if (ntok > 0x7fffffffLL || F > 0x7fffffffLL || (double)ntok * (double)F > 4.0e18 ||
+      (long long)Tg * pt > 0x7fffffffLL || (long long)Hg * ph > 0x7fffffffLL || (long long)Wg * pw > 0x7fffffffLL)
+    return VDIT_ERR_SHAPE;
+  const int esz = dtype == VDIT_F32 ? 4 : 2;
+  constexpr long long kStage = 32 * 1024;
+  if ((F + 1) * esz > kStage) return VDIT_ERR_UNSUPPORTED;
+  UnpatchifyShape s;
+  s.N = N; s.C = C; s.pt = pt; s.ph = ph; s.pw = pw; s.Tg = Tg; s.Hg = Hg; s.Wg = Wg; s.F = (int)F;
+  s.WC = (int)std::min<long long>(Wg, kStage / ((F + 1) * esz));
+  s.n_wchunks = (Wg + s.WC - 1) / s.WC;
+  const int smem = (int)((long long)s.WC * (F + 1) * esz);
+  const long long jobs = (long long)N * Tg * Hg * s.n_wchunks;
+  const long long cap = (long long)sm_count() * 8;
+  const unsigned grid = (unsigned)(jobs < cap ? jobs : cap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == VDIT_F32)
+    unpatchify3d_kernel<float><<<grid, kUnpatchifyThreads, smem, st>>>(static_cast<const float*>(tokens),
+                                                                      static_cast<float*>(latent), s);
+  else
+    unpatchify3d_kernel<__nv_bfloat16><<<grid, kUnpatchifyThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(tokens), static_cast<__nv_bfloat16*>(latent), s);
+  return last_launch_status();
+}
+
+int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bias, void* out, int N, int C, int T,
+                        int H, int W, int pt, int ph, int pw, int dim, vdit_stream_t stream) {
+  if (!latent || !weight || !out) return VDIT_ERR_NULL;
+  if (N <= 0 || C <= 0 || T <= 0 || H <= 0 || W <= 0 || pt <= 0 || ph <= 0 || pw <= 0 || dim <= 0)
+    return VDIT_ERR_SHAPE;
+  const int Tg = T / pt, Hg = H / ph, Wg = W / pw;
+  if (Tg == 0 || Hg == 0 || Wg == 0) return VDIT_ERR_SHAPE;
+  if ((long long)C * pt * ph * pw != kEmbK || dim % kEmbBN != 0) return VDIT_ERR_UNSUPPORTED;
+  if (!aligned16(weight) || !aligned16(out) || (bias && !aligned16(bias)) ||
+      (reinterpret_cast<uintptr_t>(latent) & 3u) != 0)
+    return VDIT_ERR_ALIGN;
+  const long long ntok = (long long)N * Tg * Hg * Wg;
+  if ((double)N * C * T * (double)H * W > 4.0e18 || (double)ntok * dim > 4.0e18 ||
+      (ntok + kEmbBM - 1) / kEmbBM > 0x7fffffffLL)
+    return VDIT_ERR_SHAPE;
+  static bool smem_done[kMaxDevices] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ensure_smem(patch_embed_kernel, kEmbSmem, smem_done)) return VDIT_ERR_CUDA;
+  }
+  CUtensorMap mw;
+  if (!make_2d_map(&mw, weight, kEmbK, dim, kEmbK, kEmbBN)) return VDIT_ERR_CUDA;
+  EmbedParams p;
+  p.latent = latent; p.bias = bias; p.out = static_cast<__nv_bfloat16*>(out);
+  p.C = C; p.T = T; p.H = H; p.W = W; p.pt = pt; p.ph = ph; p.pw = pw; p.Tg = Tg; p.Hg = Hg; p.Wg = Wg;
+  p.ntok = ntok; p.dim = dim;
+  p.n_mt = (int)((ntok + kEmbBM - 1) / kEmbBM);
+  const long long sms = sm_count();
+  const unsigned grid = (unsigned)(p.n_mt < sms ? p.n_mt : sms);
+  patch_embed_kernel<<<grid, kEmbThreads, kEmbSmem, reinterpret_cast<cudaStream_t>(stream)>>>(mw, p);
   return last_launch_status();
 }
 

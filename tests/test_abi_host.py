@@ -123,6 +123,32 @@ def test_cross_key_length_checked(L):
     assert attn(L, "vdit_attn_cross", dims=(1, 256, -3, 2, 128)) == SHAPE
 
 
+def embed(L, latent=FAKE, w=FAKE, b=None, out=FAKE, N=1, C=16, T=5, H=6, W=8, pt=1, ph=2, pw=2, dim=512):
+    return L.vdit_patch_embed_3d(latent, w, b, out, N, C, T, H, W, pt, ph, pw, dim, None)
+
+
+def test_patch_embed_validation(L):
+    assert embed(L, latent=None) == NULL
+    assert embed(L, w=None) == NULL
+    assert embed(L, N=0) == SHAPE
+    assert embed(L, H=1) == SHAPE                       # no whole brick along h
+    assert embed(L, C=8) == UNSUP                       # 32 features per brick
+    assert embed(L, dim=384) == UNSUP                   # not a multiple of 256
+    assert embed(L, w=MIS) == ALIGN
+    assert embed(L, b=MIS) == ALIGN
+    assert embed(L, latent=FAKE + 2) == ALIGN
+
+
+def test_unpatchify_validation(L):
+    f = lambda **kw: L.vdit_unpatchify_3d(kw.get("t", FAKE), kw.get("o", FAKE), kw.get("dt", 0), 1, 4, 2, 3, 4,
+                                          1, 2, 2, None)
+    assert f(t=None) == NULL
+    assert f(o=None) == NULL
+    assert f(dt=3) == UNSUP
+    assert L.vdit_unpatchify_3d(FAKE, FAKE, 0, 1, 4, 0, 3, 4, 1, 2, 2, None) == SHAPE
+    assert L.vdit_unpatchify_3d(FAKE, FAKE, 0, 1, 4096, 2, 3, 4, 1, 2, 2, None) == UNSUP   # 64 KB tokens
+
+
 def test_binding_refuses_cpu_tensors(L):
     """The product path has no CPU fallback: host tensors are refused."""
     import spacetime_attention_vdit_b200 as v
@@ -162,7 +188,8 @@ def test_register_budget_fits_each_sm_subpartition():
         if m and name:
             regs[name] = int(m.group(1))
     threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256,
-               "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256}
+               "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256, "patch_embed_kernel": 320,
+               "unpatchify3d_kernel": 256}
 
     def block_of(kname):
         for key, t in threads.items():
