@@ -21,9 +21,10 @@ namespace vdit {
 //
 // One CTA per run of WC bricks that share (n, t', h'): their tokens are one
 // contiguous span of WC*F elements, copied to shared memory with a padded
-// stride (F + 1: the lanes that gather one latent row read different banks);
-// then the C*pt*ph latent rows they fill (each WC*pw elements along w) are
-// written with coalesced stores.
+// stride (F + 1: the lanes that read one latent row's values from consecutive
+// tokens hit different banks), with 16-byte loads when aligned; then one thread
+// per (latent row, brick) writes the brick's pw values of that row, so that
+// neighbouring lanes store neighbouring addresses.
 
 struct UnpatchifyShape {
   int N, C, pt, ph, pw;
@@ -35,9 +36,14 @@ struct UnpatchifyShape {
 
 constexpr int kUnpatchifyThreads = 256;
 
+template <typename E> struct Pair;
+template <> struct Pair<float> { using type = float2; };
+template <> struct Pair<__nv_bfloat16> { using type = __nv_bfloat162; };
+
 template <typename E>
 __global__ void __launch_bounds__(kUnpatchifyThreads) unpatchify3d_kernel(const E* __restrict__ tokens,
-                                                                         E* __restrict__ latent, UnpatchifyShape s) {
+                                                                         E* __restrict__ latent, UnpatchifyShape s,
+                                                                         bool vec_in, bool pair_out) {
   E* stage = reinterpret_cast<E*>(dyn_smem);
   if (watchdog_tripped()) return;
   const int T = s.Tg * s.pt, H = s.Hg * s.ph, W = s.Wg * s.pw;
@@ -54,21 +60,43 @@ __global__ void __launch_bounds__(kUnpatchifyThreads) unpatchify3d_kernel(const 
     const int nb = min(s.WC, s.Wg - w0);
     const E* src = tokens + ((((long long)n * s.Tg + tq) * s.Hg + hq) * s.Wg + w0) * s.F;
     __syncthreads();
-    for (int e = threadIdx.x; e < nb * s.F; e += blockDim.x) {
-      const int b = e / s.F, f = e - b * s.F;
-      stage[b * rs + f] = src[e];
+    if (vec_in) {                                           // 16-byte loads, 16 / sizeof(E) elements each
+      constexpr int V = 16 / sizeof(E);
+      const int n4 = nb * s.F / V;
+      for (int e4 = threadIdx.x; e4 < n4; e4 += blockDim.x) {
+        const uint4 u = reinterpret_cast<const uint4*>(src)[e4];
+        const E* ue = reinterpret_cast<const E*>(&u);
+        const int e = e4 * V, b = e / s.F, f = e - b * s.F;   // F is a multiple of V: one token
+#pragma unroll
+        for (int m = 0; m < V; ++m) stage[b * rs + f + m] = ue[m];
+      }
+    } else {
+      for (int e = threadIdx.x; e < nb * s.F; e += blockDim.x) {
+        const int b = e / s.F, f = e - b * s.F;
+        stage[b * rs + f] = src[e];
+      }
     }
     __syncthreads();
-    const int len = nb * s.pw;                             // elements of each latent row written
+    // one thread per (latent row (c, dt, dh), brick b): the brick's pw values of
+    // the row, which are consecutive features of the token; neighbouring lanes
+    // take neighbouring bricks, so the stores are contiguous
     const int nrows = s.C * s.pt * s.ph;
-    for (int e = threadIdx.x; e < nrows * len; e += blockDim.x) {
-      const int row = e / len, x = e - row * len;          // row = (c, dt, dh)
+    for (int e = threadIdx.x; e < nrows * nb; e += blockDim.x) {
+      const int row = e / nb, b = e - row * nb;
       const int dh = row % s.ph, cdt = row / s.ph;
       const int dt = cdt % s.pt, c = cdt / s.pt;
-      const int b = x / s.pw, dw = x - b * s.pw;
-      const int f = ((c * s.pt + dt) * s.ph + dh) * s.pw + dw;
-      latent[(((long long)n * s.C + c) * T + tq * s.pt + dt) * ((long long)H * W) +
-             (long long)(hq * s.ph + dh) * W + w0 * s.pw + x] = stage[b * rs + f];
+      const int f0 = ((c * s.pt + dt) * s.ph + dh) * s.pw;
+      E* dst = latent + (((long long)n * s.C + c) * T + tq * s.pt + dt) * ((long long)H * W) +
+               (long long)(hq * s.ph + dh) * W + (long long)(w0 + b) * s.pw;
+      const E* sp = stage + b * rs + f0;
+      if (pair_out) {                                       // pw == 2: one 2-element store
+        typename Pair<E>::type v;
+        v.x = sp[0];
+        v.y = sp[1];
+        *reinterpret_cast<typename Pair<E>::type*>(dst) = v;
+      } else {
+        for (int dw = 0; dw < s.pw; ++dw) dst[dw] = sp[dw];
+      }
     }
   }
 }
@@ -91,8 +119,11 @@ __global__ void __launch_bounds__(kUnpatchifyThreads) unpatchify3d_kernel(const 
 //               bf16 and writes the 128-byte row in the swizzled layout (two
 //               A buffers, so the next tile is gathered during this one's
 //               products);
-//   warps 2..5  epilogue: accumulator + bias, rounded to bf16, stored; one
-//               thread per token row (TMEM lane = row), 16-byte stores.
+//   warps 2..5  epilogue: accumulator + bias, rounded to bf16; one thread per
+//               token row (TMEM lane = row).  Each warp writes its 32 rows of a
+//               64-column box into a staging buffer of its own (128-byte
+//               swizzle) and lane 0 sends it out with a TMA store, so the
+//               stores are whole lines and the warps never wait on each other.
 // Every wait is bounded by the watchdog; copies and UMMAs are drained before
 // the CTA exits.
 
@@ -101,7 +132,10 @@ constexpr int kEmbNW = 3;                                  // weight ring stages
 constexpr int kEmbThreads = 320;
 constexpr int kEmbATile = kEmbBM * kEmbK * 2;              // 16 KB
 constexpr int kEmbWTile = kEmbBN * kEmbK * 2;              // 32 KB
-constexpr int kEmbSmem = 1024 + 2 * kEmbATile + kEmbNW * kEmbWTile + 256 + kEmbK * 4;
+constexpr int kEmbOutBox = 64;                              // output columns per TMA store box
+constexpr int kEmbStage = 32 * kEmbOutBox * 2;             // one warp's box: 32 rows x 128 bytes
+constexpr int kEmbNStage = 4;                              // staging boxes per warp
+constexpr int kEmbSmem = 1024 + 2 * kEmbATile + kEmbNW * kEmbWTile + 4 * kEmbNStage * kEmbStage + 256 + kEmbK * 4;
 constexpr uint32_t kEmbIdesc = umma_idesc_bf16(kEmbBM, kEmbBN, 0, 0);
 
 struct EmbedParams {
@@ -117,11 +151,13 @@ struct EmbedParams {
 enum : int { kSiteEmbA = 40, kSiteEmbW, kSiteEmbAcc, kSiteEmbDrain };
 
 __global__ void __launch_bounds__(kEmbThreads, 1)
-    patch_embed_kernel(const __grid_constant__ CUtensorMap tmW, const EmbedParams p) {
+    patch_embed_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmOut,
+                       const EmbedParams p) {
   const uintptr_t base = (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023);
   unsigned char* sA = reinterpret_cast<unsigned char*>(base);            // 2 A buffers
   unsigned char* sW = sA + 2 * kEmbATile;                                // weight ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + kEmbNW * kEmbWTile);
+  unsigned char* sOut = sW + kEmbNW * kEmbWTile;                       // [epilogue warp][kEmbNStage] boxes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 4 * kEmbNStage * kEmbStage);
   uint64_t* a_full = bars;            // [2] the gather warps filled the buffer
   uint64_t* a_empty = a_full + 2;     // [2] the buffer's UMMAs finished
   uint64_t* w_full = a_empty + 2;     // [kEmbNW]
@@ -250,21 +286,28 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    unsigned char* my_stage = sOut + quad * kEmbNStage * kEmbStage;
+    int boxes = 0;                                      // boxes this warp has sent
     for (int lt = 0; lt < n_my; ++lt) {
-      const long long tok = ((long long)blockIdx.x + (long long)lt * gridDim.x) * kEmbBM + r;
+      const long long tile0 = ((long long)blockIdx.x + (long long)lt * gridDim.x) * kEmbBM;
       bool ok = true;
       for (int nt = 0; nt < n_nt; ++nt) {
         const int st = lt * n_nt + nt, ac = st & 1;
         if (!warp_wait(&acc_full[ac], (st >> 1) & 1, kSiteEmbAcc)) { ok = false; break; }
         tc_fence_after();
-        __nv_bfloat16* orow = p.out + tok * p.dim + nt * kEmbBN;
 #pragma unroll 1
-        for (int c = 0; c < kEmbBN / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tl + ac * kEmbBN + c * 32, o);
-          tmem_ld_wait();
-          if (tok < p.ntok) {
-            const int col = nt * kEmbBN + c * 32;
+        for (int bx = 0; bx < kEmbBN / kEmbOutBox; ++bx, ++boxes) {
+          unsigned char* box = my_stage + (boxes % kEmbNStage) * kEmbStage;
+          if (boxes >= kEmbNStage) {                    // the TMA store that used this buffer has read it
+            if (lane == 0) bulk_wait_group_read<kEmbNStage - 1>();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int h = 0; h < kEmbOutBox / 32; ++h) {
+            uint32_t o[32];
+            tmem_ld32(tl + ac * kEmbBN + bx * kEmbOutBox + h * 32, o);
+            tmem_ld_wait();
+            const int col = nt * kEmbBN + bx * kEmbOutBox + h * 32;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               float b8[8];
@@ -282,8 +325,15 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
               v.y = pack_bf16x2(__uint_as_float(o[e + 2]) + b8[2], __uint_as_float(o[e + 3]) + b8[3]);
               v.z = pack_bf16x2(__uint_as_float(o[e + 4]) + b8[4], __uint_as_float(o[e + 5]) + b8[5]);
               v.w = pack_bf16x2(__uint_as_float(o[e + 6]) + b8[6], __uint_as_float(o[e + 7]) + b8[7]);
-              *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+              const int j = h * 4 + e / 8;              // 16-byte chunk of the 128-byte row
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
             }
+          }
+          fence_proxy_async_smem();                     // the TMA engine reads what the lanes wrote
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, box, nt * kEmbBN + bx * kEmbOutBox, (int)(tile0 + quad * 32));
+            bulk_commit_group();
           }
         }
         tc_fence_before();
@@ -292,6 +342,8 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
       }
       if (!ok) break;
     }
+    if (lane == 0) bulk_wait_group_all();               // every store has landed before the CTA exits
+    (void)r;
   }
 
   tc_fence_before();

@@ -335,12 +335,17 @@ int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C
   const long long cap = (long long)sm_count() * 8;
   const unsigned grid = (unsigned)(jobs < cap ? jobs : cap);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // 16-byte loads when every token starts 16-byte aligned; paired stores when
+  // pw == 2 and every brick's pair is aligned (W = Wg * 2 is even)
+  const bool vec_in = aligned16(tokens) && (F * esz) % 16 == 0;
+  const bool pair_out = pw == 2 && (reinterpret_cast<uintptr_t>(latent) % (2 * esz)) == 0;
   if (dtype == VDIT_F32)
     unpatchify3d_kernel<float><<<grid, kUnpatchifyThreads, smem, st>>>(static_cast<const float*>(tokens),
-                                                                      static_cast<float*>(latent), s);
+                                                                      static_cast<float*>(latent), s, vec_in,
+                                                                      pair_out);
   else
     unpatchify3d_kernel<__nv_bfloat16><<<grid, kUnpatchifyThreads, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(tokens), static_cast<__nv_bfloat16*>(latent), s);
+        static_cast<const __nv_bfloat16*>(tokens), static_cast<__nv_bfloat16*>(latent), s, vec_in, pair_out);
   return last_launch_status();
 }
 
@@ -365,8 +370,9 @@ int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bi
     std::lock_guard<std::mutex> lock(mu);
     if (!ensure_smem(patch_embed_kernel, kEmbSmem, smem_done)) return VDIT_ERR_CUDA;
   }
-  CUtensorMap mw;
-  if (!make_2d_map(&mw, weight, kEmbK, dim, kEmbK, kEmbBN)) return VDIT_ERR_CUDA;
+  CUtensorMap mw, mo;
+  if (!make_2d_map(&mw, weight, kEmbK, dim, kEmbK, kEmbBN) || !make_2d_map(&mo, out, dim, ntok, kEmbOutBox, 32))
+    return VDIT_ERR_CUDA;
   EmbedParams p;
   p.latent = latent; p.bias = bias; p.out = static_cast<__nv_bfloat16*>(out);
   p.C = C; p.T = T; p.H = H; p.W = W; p.pt = pt; p.ph = ph; p.pw = pw; p.Tg = Tg; p.Hg = Hg; p.Wg = Wg;
@@ -374,7 +380,7 @@ int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bi
   p.n_mt = (int)((ntok + kEmbBM - 1) / kEmbBM);
   const long long sms = sm_count();
   const unsigned grid = (unsigned)(p.n_mt < sms ? p.n_mt : sms);
-  patch_embed_kernel<<<grid, kEmbThreads, kEmbSmem, reinterpret_cast<cudaStream_t>(stream)>>>(mw, p);
+  patch_embed_kernel<<<grid, kEmbThreads, kEmbSmem, reinterpret_cast<cudaStream_t>(stream)>>>(mw, mo, p);
   return last_launch_status();
 }
 
