@@ -77,25 +77,28 @@ __global__ void __launch_bounds__(kUnpatchifyThreads) unpatchify3d_kernel(const 
       }
     }
     __syncthreads();
-    // one thread per (latent row (c, dt, dh), brick b): the brick's pw values of
-    // the row, which are consecutive features of the token; neighbouring lanes
-    // take neighbouring bricks, so the stores are contiguous
+    // one warp per latent row (c, dt, dh), one lane per brick: the brick's pw
+    // values of the row, which are consecutive features of the token;
+    // neighbouring lanes take neighbouring bricks, so the stores are contiguous
     const int nrows = s.C * s.pt * s.ph;
-    for (int e = threadIdx.x; e < nrows * nb; e += blockDim.x) {
-      const int row = e / nb, b = e - row * nb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    for (int row = warp; row < nrows; row += nwarps) {   // row = (c, dt, dh)
       const int dh = row % s.ph, cdt = row / s.ph;
       const int dt = cdt % s.pt, c = cdt / s.pt;
       const int f0 = ((c * s.pt + dt) * s.ph + dh) * s.pw;
-      E* dst = latent + (((long long)n * s.C + c) * T + tq * s.pt + dt) * ((long long)H * W) +
-               (long long)(hq * s.ph + dh) * W + (long long)(w0 + b) * s.pw;
-      const E* sp = stage + b * rs + f0;
-      if (pair_out) {                                       // pw == 2: one 2-element store
-        typename Pair<E>::type v;
-        v.x = sp[0];
-        v.y = sp[1];
-        *reinterpret_cast<typename Pair<E>::type*>(dst) = v;
-      } else {
-        for (int dw = 0; dw < s.pw; ++dw) dst[dw] = sp[dw];
+      E* drow = latent + (((long long)n * s.C + c) * T + tq * s.pt + dt) * ((long long)H * W) +
+                (long long)(hq * s.ph + dh) * W + (long long)w0 * s.pw;
+      for (int b = lane; b < nb; b += 32) {
+        const E* sp = stage + b * rs + f0;
+        E* dst = drow + (long long)b * s.pw;
+        if (pair_out) {                                   // pw == 2: one 2-element store
+          typename Pair<E>::type v;
+          v.x = sp[0];
+          v.y = sp[1];
+          *reinterpret_cast<typename Pair<E>::type*>(dst) = v;
+        } else {
+          for (int dw = 0; dw < s.pw; ++dw) dst[dw] = sp[dw];
+        }
       }
     }
   }
@@ -146,6 +149,9 @@ struct EmbedParams {
   long long ntok;            // N * L
   int dim;                   // model width, a multiple of 256
   int n_mt;                  // token tiles
+  int group_nt;              // N tiles per work item
+  int n_groups;              // work items per token tile
+  int n_items;               // n_mt * n_groups
 };
 
 enum : int { kSiteEmbA = 40, kSiteEmbW, kSiteEmbAcc, kSiteEmbDrain };
@@ -170,7 +176,14 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_nt = p.dim / kEmbBN;
-  const int n_my = (int)blockIdx.x < p.n_mt ? (p.n_mt - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // Work item w = (token tile w / n_groups, N tiles [g G, g G + G) with g = w mod
+  // n_groups): CTA c takes items c, c + gridDim.x, ...  Splitting a token tile's
+  // N tiles over several items keeps the last wave of CTAs short.
+  const int n_my = (int)blockIdx.x < p.n_items ? (p.n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto item_w = [&](int lt) { return (int)blockIdx.x + lt * (int)gridDim.x; };
+  auto item_tm = [&](int lt) { return item_w(lt) / p.n_groups; };
+  auto item_nt0 = [&](int lt) { return (item_w(lt) % p.n_groups) * p.group_nt; };
+  auto item_nn = [&](int lt) { return min(p.group_nt, n_nt - item_nt0(lt)); };
   const long long plane = (long long)p.H * p.W;
 
   if (threadIdx.x == 0) {
@@ -203,14 +216,17 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       tma_prefetch_desc(&tmW);
-      const int steps = n_my * n_nt;
       int issued = 0;
-      for (int st = 0; st < steps; ++st) {
-        const int s = st % kEmbNW;
-        if (st >= kEmbNW && !mbar_wait(&w_empty[s], ((st / kEmbNW) - 1) & 1, kSiteEmbW)) break;
-        mbar_arrive_expect_tx(&w_full[s], kEmbWTile);
-        tma_load_2d(sW + s * kEmbWTile, &tmW, &w_full[s], 0, (st % n_nt) * kEmbBN);
-        ++issued;
+      bool ok = true;
+      for (int lt = 0; lt < n_my && ok; ++lt) {
+        const int nt0 = item_nt0(lt), nn = item_nn(lt);
+        for (int j = 0; j < nn; ++j) {
+          const int st = issued, s = st % kEmbNW;
+          if (st >= kEmbNW && !mbar_wait(&w_empty[s], ((st / kEmbNW) - 1) & 1, kSiteEmbW)) { ok = false; break; }
+          mbar_arrive_expect_tx(&w_full[s], kEmbWTile);
+          tma_load_2d(sW + s * kEmbWTile, &tmW, &w_full[s], 0, (nt0 + j) * kEmbBN);
+          ++issued;
+        }
       }
       for (int st = issued - kEmbNW < 0 ? 0 : issued - kEmbNW; st < issued; ++st)
         mbar_drain_site(&w_full[st % kEmbNW], (st / kEmbNW) & 1, kSiteEmbDrain);
@@ -220,11 +236,13 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
     if (lane == 0) {
       const uint32_t sAa = smem_u32(sA), sWa = smem_u32(sW);
       bool ok = true;
+      int st = 0;                                       // N tiles done by this CTA
       for (int lt = 0; lt < n_my && ok; ++lt) {
         const int ab = lt & 1;
         if (!mbar_wait(&a_full[ab], (lt >> 1) & 1, kSiteEmbA)) { ok = false; break; }
-        for (int nt = 0; nt < n_nt && ok; ++nt) {
-          const int st = lt * n_nt + nt, s = st % kEmbNW, ac = st & 1;
+        const int nn = item_nn(lt);
+        for (int j = 0; j < nn && ok; ++j, ++st) {
+          const int s = st % kEmbNW, ac = st & 1;
           if (!mbar_wait(&w_full[s], (st / kEmbNW) & 1, kSiteEmbW) ||
               (st >= 2 && !mbar_wait(&acc_empty[ac], ((st >> 1) - 1) & 1, kSiteEmbAcc))) {
             ok = false;
@@ -252,7 +270,7 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
     for (int lt = 0; lt < n_my; ++lt) {
       const int ab = lt & 1;
       if (lt >= 2 && !warp_wait(&a_empty[ab], ((lt >> 1) - 1) & 1, kSiteEmbA)) break;
-      const long long tok = ((long long)blockIdx.x + (long long)lt * gridDim.x) * kEmbBM + r;
+      const long long tok = (long long)item_tm(lt) * kEmbBM + r;
       unsigned char* row = sA + ab * kEmbATile + r * 128;
       if (tok < p.ntok) {
         long long q = tok;
@@ -288,11 +306,13 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     unsigned char* my_stage = sOut + quad * kEmbNStage * kEmbStage;
     int boxes = 0;                                      // boxes this warp has sent
+    int st = 0;                                         // N tiles done by this CTA
     for (int lt = 0; lt < n_my; ++lt) {
-      const long long tile0 = ((long long)blockIdx.x + (long long)lt * gridDim.x) * kEmbBM;
+      const long long tile0 = (long long)item_tm(lt) * kEmbBM;
+      const int nt0 = item_nt0(lt), nn = item_nn(lt);
       bool ok = true;
-      for (int nt = 0; nt < n_nt; ++nt) {
-        const int st = lt * n_nt + nt, ac = st & 1;
+      for (int j = 0; j < nn; ++j, ++st) {
+        const int nt = nt0 + j, ac = st & 1;
         if (!warp_wait(&acc_full[ac], (st >> 1) & 1, kSiteEmbAcc)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1

@@ -378,8 +378,13 @@ int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bi
   p.C = C; p.T = T; p.H = H; p.W = W; p.pt = pt; p.ph = ph; p.pw = pw; p.Tg = Tg; p.Hg = Hg; p.Wg = Wg;
   p.ntok = ntok; p.dim = dim;
   p.n_mt = (int)((ntok + kEmbBM - 1) / kEmbBM);
+  const int n_nt = dim / kEmbBN;
+  p.group_nt = (n_nt + 3) / 4;                         // up to four work items per token tile
+  p.n_groups = (n_nt + p.group_nt - 1) / p.group_nt;
+  if ((long long)p.n_mt * p.n_groups > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  p.n_items = p.n_mt * p.n_groups;
   const long long sms = sm_count();
-  const unsigned grid = (unsigned)(p.n_mt < sms ? p.n_mt : sms);
+  const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
   patch_embed_kernel<<<grid, kEmbThreads, kEmbSmem, reinterpret_cast<cudaStream_t>(stream)>>>(mw, mo, p);
   return last_launch_status();
 }
