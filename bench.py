@@ -416,7 +416,7 @@ def main():
                 last.record(s_out)
 
         run_pipeline(2)
-        e_steps = max(4, min(args.steps, 8))
+        e_steps = max(4, min(args.steps, 16))
         barrier()
         torch.cuda.synchronize(dev)
         s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
