@@ -187,7 +187,10 @@ def oracle_sample(d, budget_s, seed=0):
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-        rows = min(4096, rows * 2)
+        # the next chunk: at most double, and no longer than the time left at the
+        # rate just measured, so a step stays close to its budget
+        per_row = el / done_rows
+        rows = int(max(16, min(4096, rows * 2, (budget_s - el) / per_row + 1)))
     return flops, el, f"{done_rows} query rows of one (batch, head): full attention over all {L} keys, " \
                       f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy"
 
