@@ -25,7 +25,8 @@ def L():
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "vdit.h")).read()
+    with open(os.path.join(ROOT, "include", "vdit.h")) as fh:
+        text = fh.read()
     return sorted(set(re.findall(r"^(?:int|const char\*)\s+(vdit_\w+)\s*\(", text, flags=re.M)))
 
 

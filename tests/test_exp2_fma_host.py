@@ -15,7 +15,8 @@ SRC = os.path.join(ROOT, "spacetime_attention_vdit_b200", "csrc", "attn_tcgen05.
 
 
 def coefficients():
-    text = open(SRC).read()
+    with open(SRC) as fh:
+        text = fh.read()
     body = text[text.index("float2 ex2_fma2(float2 x)"):]
     body = body[:body.index("\n}\n")]
     c3 = float(re.search(r"make_float2\(([0-9.e+-]+)f, \1f\), f, make_float2\(([0-9.e+-]+)f", body).group(1))

@@ -68,7 +68,7 @@ def _rank_main(rank, world, port, out):
 
 @pytest.mark.parametrize("world", [2, 4])
 def test_ulysses_gloo(world):
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     for r in range(world):
