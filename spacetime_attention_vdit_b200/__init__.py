@@ -11,10 +11,14 @@ passes none).
 Calls (see ``include/vdit.h`` for the exact definitions and sources):
 
 * :func:`patchify_3d`         latent [N, C, T, H, W] -> tokens [N, L, C*pt*ph*pw]
+* :func:`patch_embed_3d`      the Conv3d patch embedding: tokens @ weight^T + bias
+* :func:`unpatchify_3d`       tokens [N, L, C*pt*ph*pw] -> latent [N, C, T, H, W]
 * :func:`rope_3d`             3D rotary positions on Q and K [B, L, heads, D]
+* :func:`qk_norm_rope_3d`     RMSNorm of Q and K, then the 3D rotation, in one pass
 * :func:`attn_full`           full 3D self-attention
 * :func:`attn_divided_time`   attention over the T tokens of each spatial site
 * :func:`attn_divided_space`  attention over the HW tokens of each frame
+* :func:`attn_cross`          video tokens attending to a separate key/value sequence
 """
 from __future__ import annotations
 
@@ -23,8 +27,9 @@ import os
 
 import torch
 
-__all__ = ["VditError", "lib", "patchify_3d", "patch_embed_3d", "unpatchify_3d", "rope_3d", "qk_norm_rope_3d", "attn_full", "attn_divided_time",
-           "attn_divided_space", "attn_cross", "device_status", "status_string", "default_split", "LIB_PATH"]
+__all__ = ["VditError", "lib", "patchify_3d", "patch_embed_3d", "unpatchify_3d", "rope_3d",
+           "qk_norm_rope_3d", "attn_full", "attn_divided_time", "attn_divided_space", "attn_cross",
+           "device_status", "status_string", "default_split", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
 
