@@ -9,49 +9,66 @@
 // about 10 flop/byte: it is bandwidth-bound, and is built to keep HBM busy.
 //
 // Design: a producer warp streams problems into a ring of shared-memory stages
-// with TMA - one 5-D box per D-block per tensor: {D-block, 1 head, 1 site, TP
+// with TMA - one 5-D box per D-block per tensor: {D-block, 1 head, 1 site, TB
 // frames, 1 batch} over the view {D, heads, sites, frames, batch}, so the box
 // gathers the site's T rows (HW*heads*D elements apart) in one copy and rows
-// TP > T arrive as zeros.  Each consumer group (two warps when T > 16, one per
-// 16-row m-tile; one warp otherwise) owns two stages and alternates between
-// them, so its next problem is in flight while it computes the current one.
-// A consumer warp computes S = Q K^T and O = P V with warp-level bf16
-// tensor-core MMAs (m16n8k16, fp32 accumulation) on rows padded to TP, keeps the
-// softmax in registers, stages O over the stage's Q rows and writes it with
-// 16-byte stores, then releases the stage to the producer.
+// T .. TB-1 arrive as zeros.  TB is T rounded up to 8 rows, so that as many
+// problems as possible fit in shared memory at once (at T = 21, 24-row stages
+// hold 10 problems where 32-row ones held 8).  Each consumer group (two warps
+// when T > 16, one per 16-row m-tile; one warp otherwise) owns two stages and
+// alternates between them, so its next problem is in flight while it computes
+// the current one.  A consumer warp computes S = Q K^T and O = P V with
+// warp-level bf16 tensor-core MMAs (m16n8k16, fp32 accumulation) on rows padded
+// to TP (TB rounded up to 16; the rows TB .. TP-1 that a fragment load reaches
+// read rows TB-8 .. TP-9 again: their scores are masked, their probabilities
+// are exactly zero and their query rows are never stored), keeps the softmax in
+// registers, stages O over the stage's Q rows and writes it with 16-byte
+// stores, then releases the stage to the producer.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace vdit {
 
-template <int D, int TP>
+template <int D, int TB>
 struct TimeCfg {
+  static constexpr int TP = (TB + 15) & ~15;                  // rows and keys padded to 16-row m-tiles
   static constexpr int ROWB = (D * 2 >= 128) ? 128 : D * 2;   // bytes per row of one D-block
   static constexpr int DBLK = ROWB / 2;                       // elements per D-block
   static constexpr int NDB = D / DBLK;                        // D-blocks
   static constexpr int CPB = ROWB / 16;                       // 16-byte chunks per D-block row
-  static constexpr int REGION = TP * ROWB;                    // one D-block of one tensor
-  static constexpr int TENSOR_BYTES = NDB * REGION;           // = TP * D * 2
+  static constexpr int REGION = TB * ROWB;                    // one D-block of one tensor
+  static constexpr int TENSOR_BYTES = NDB * REGION;           // = TB * D * 2
   static constexpr int STAGE_BYTES = 3 * TENSOR_BYTES;        // Q, K, V
-  static constexpr int NSTAGE_MAX = (196608 / STAGE_BYTES) & ~1;
-  static constexpr int NSTAGE = NSTAGE_MAX > 16 ? 16 : NSTAGE_MAX;
-  static constexpr int NP = NSTAGE / 2;                       // consumer groups, two stages each
   static constexpr int WPU = TP >= 32 ? 2 : 1;                // warps per problem (split by 16-row m-tiles)
+  // stages: as many as fit in the 227 KB a CTA may use, at most 16, and at most
+  // 10 consumer warps at D = 128 so that the registers of the fullest SM
+  // sub-partition (three warps of eleven) stay within its 16,384
+  static constexpr int MAXW = D >= 128 ? 10 : 16;
+  static constexpr int FIT = (231424 / (STAGE_BYTES + 16)) & ~1;
+  static constexpr int NSTAGE = FIT < 16 ? (FIT < 2 * (MAXW / WPU) ? FIT : 2 * (MAXW / WPU))
+                                         : (16 < 2 * (MAXW / WPU) ? 16 : 2 * (MAXW / WPU));
+  static constexpr int NP = NSTAGE / 2;                       // consumer groups, two stages each
   static constexpr int NC = NP * WPU;                         // consumer warps
   static constexpr int THREADS = 32 * (1 + NC);
+  // register budget as if the warps filled every sub-partition evenly
+  static constexpr int LB_THREADS = 128 * ((1 + NC + 3) / 4);
   static constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 2 * NSTAGE * 8;
   static_assert(D % 16 == 0 && D >= 32 && D <= 128, "head_dim");
-  static_assert(TP == 16 || TP == 32 || TP == 64, "padded length");
+  static_assert(TB % 8 == 0 && TB >= 8 && TB <= 64, "box rows");
   static_assert(NSTAGE >= 2, "stages");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 // Byte offset of 16-byte chunk c (0 .. D/8-1) of row r inside one tensor of a
 // stage, as the TMA box lays it out: D-block c / CPB, rows of ROWB bytes, the
-// chunk index XOR-swizzled with the row (128-byte or 64-byte swizzle).
-template <int D, int TP>
+// chunk index XOR-swizzled with the row (128-byte or 64-byte swizzle).  Rows
+// TB .. TP-1 (only when TB is not a multiple of 16) fold back by 8 onto rows
+// that the stage holds.
+template <int D, int TB>
 __device__ __forceinline__ uint32_t time_off(int r, int c) {
-  using C = TimeCfg<D, TP>;
+  using C = TimeCfg<D, TB>;
+  if (TB != C::TP && r >= TB) r -= 8;
   const int key = C::ROWB == 128 ? (r & 7) : ((r >> 1) & 3);
   return (uint32_t)((c / C::CPB) * C::REGION + r * C::ROWB + (((c % C::CPB) ^ key) << 4));
 }
@@ -82,11 +99,12 @@ struct TimeParams {
   float scale_log2;
 };
 
-template <int D, int TP>
-__global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
+template <int D, int TB>
+__global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
     attn_time_short_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const TimeParams p) {
-  using C = TimeCfg<D, TP>;
+  using C = TimeCfg<D, TB>;
+  constexpr int TP = C::TP;
   const uintptr_t base = (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023);
   unsigned char* stages = reinterpret_cast<unsigned char*>(base);
   uint64_t* full = reinterpret_cast<uint64_t*>(stages + C::NSTAGE * C::STAGE_BYTES);
@@ -172,11 +190,11 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(aQ + time_off<D, TP>(mt * 16 + (lane & 15), kk * 2 + (lane >> 4)), a0, a1, a2, a3);
+        ldsm_x4(aQ + time_off<D, TB>(mt * 16 + (lane & 15), kk * 2 + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
         for (int np = 0; np < TP / 16; ++np) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(aK + time_off<D, TP>(np * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)),
+          ldsm_x4(aK + time_off<D, TB>(np * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)),
                   b0, b1, b2, b3);
           mma_bf16_16816(sacc[2 * np], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(sacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
@@ -227,7 +245,7 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
 #pragma unroll
         for (int dp = 0; dp < D / 16; ++dp) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(aV + time_off<D, TP>(k2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), dp * 2 + (lane >> 4)),
+          ldsm_x4_t(aV + time_off<D, TB>(k2 * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), dp * 2 + (lane >> 4)),
                     b0, b1, b2, b3);
           mma_bf16_16816(oacc[2 * dp], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(oacc[2 * dp + 1], a0, a1, a2, a3, b2, b3);
@@ -240,10 +258,10 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
 #pragma unroll
       for (int n = 0; n < D / 8; ++n) {       // 8 columns = one 16-byte chunk
         if (r0 < T)
-          *reinterpret_cast<uint32_t*>(sb + time_off<D, TP>(r0, n) + q2 * 2) =
+          *reinterpret_cast<uint32_t*>(sb + time_off<D, TB>(r0, n) + q2 * 2) =
               pack_bf16x2(oacc[n][0] * inv0, oacc[n][1] * inv0);
         if (r1 < T)
-          *reinterpret_cast<uint32_t*>(sb + time_off<D, TP>(r1, n) + q2 * 2) =
+          *reinterpret_cast<uint32_t*>(sb + time_off<D, TB>(r1, n) + q2 * 2) =
               pack_bf16x2(oacc[n][2] * inv1, oacc[n][3] * inv1);
       }
       if (p.lse != nullptr && (lane & 3) == 0) {
@@ -260,7 +278,7 @@ __global__ void __launch_bounds__(TimeCfg<D, TP>::THREADS, 1)
       const int rows = min(16, T - mt * 16);
       for (int i = lane; i < rows * (D / 8); i += 32) {
         const int t = mt * 16 + i / (D / 8), c = i % (D / 8);
-        const uint4 val = *reinterpret_cast<const uint4*>(sb + time_off<D, TP>(t, c));
+        const uint4 val = *reinterpret_cast<const uint4*>(sb + time_off<D, TB>(t, c));
         *reinterpret_cast<uint4*>(p.o + first + t * row_stride + c * 8) = val;
       }
     }

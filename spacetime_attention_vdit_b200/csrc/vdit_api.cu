@@ -174,35 +174,38 @@ int dispatch_tcgen05(int D, const void* q, const void* k, const void* v, void* o
   }
 }
 
-template <int D, int TP>
+template <int D, int TB>
 int launch_time_short(const void* q, const void* k, const void* v, const TimeParams& p, cudaStream_t stream) {
-  using C = TimeCfg<D, TP>;
+  using C = TimeCfg<D, TB>;
   static bool smem_done[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (!ensure_smem(attn_time_short_kernel<D, TP>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
+    if (!ensure_smem(attn_time_short_kernel<D, TB>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
   }
-  // view {D, heads, sites, frames, batch}; one box = one site's TP frames of one head
+  // view {D, heads, sites, frames, batch}; one box = one site's TB frames of one head
   const long long tok = (long long)p.heads * D;
   CUtensorMap mq, mk, mv;
   const long long site_st = tok, frame_st = tok * p.HW, batch_st = tok * p.HW * p.T;
-  if (!make_qkv_map(&mq, q, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP) ||
-      !make_qkv_map(&mk, k, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP) ||
-      !make_qkv_map(&mv, v, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TP))
+  if (!make_qkv_map(&mq, q, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TB) ||
+      !make_qkv_map(&mk, k, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TB) ||
+      !make_qkv_map(&mv, v, D, p.heads, p.HW, p.T, p.B, site_st, frame_st, batch_st, TB))
     return VDIT_ERR_CUDA;
   const long long units = (long long)p.B * p.HW * p.heads;
   const long long cap = (long long)sm_count();       // one persistent CTA per SM
   const unsigned grid = (unsigned)(units < cap ? units : cap);
-  attn_time_short_kernel<D, TP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  attn_time_short_kernel<D, TB><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return last_launch_status();
 }
 
 template <int D>
 int dispatch_time_short_tp(const void* q, const void* k, const void* v, const TimeParams& p,
                            cudaStream_t stream) {
+  // box rows: T rounded up to 8 (16 at least), from the set compiled here
   if (p.T <= 16) return launch_time_short<D, 16>(q, k, v, p, stream);
+  if (p.T <= 24) return launch_time_short<D, 24>(q, k, v, p, stream);
   if (p.T <= 32) return launch_time_short<D, 32>(q, k, v, p, stream);
+  if (p.T <= 48) return launch_time_short<D, 48>(q, k, v, p, stream);
   return launch_time_short<D, 64>(q, k, v, p, stream);
 }
 

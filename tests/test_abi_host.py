@@ -197,10 +197,12 @@ def test_register_budget_fits_each_sm_subpartition():
             if key in kname:
                 return t
         m = re.search(r"attn_time_short_kernelILi(\d+)ELi(\d+)", kname)
-        D, TP = int(m.group(1)), int(m.group(2))
-        stage = 3 * TP * D * 2
-        nstage = min(16, (196608 // stage) & ~1)
-        wpu = 2 if TP >= 32 else 1
+        D, TB = int(m.group(1)), int(m.group(2))       # head dim, box rows
+        tp = (TB + 15) // 16 * 16
+        wpu = 2 if tp >= 32 else 1
+        stage = 3 * TB * D * 2
+        nstage = min((231424 // (stage + 16)) & ~1, 16, 2 * ((10 if D >= 128 else 16) // wpu))
+        assert 1024 + nstage * (stage + 16) <= 232448
         return 32 * (1 + (nstage // 2) * wpu)
     assert regs, "no ptxas report"
     for kname, r in regs.items():

@@ -128,10 +128,15 @@ def test_full_constant_keys():
     (8, 64, 2, 32),
     (16, 9, 2, 128),
     (17, 7, 3, 128),
-    (21, 13, 2, 128),      # the 81-frame latent length
+    (21, 13, 2, 128),      # the 81-frame latent length (24-row boxes)
     (21, 6, 1, 64),
+    (23, 4, 2, 32),
+    (24, 5, 2, 128),
+    (25, 3, 2, 64),
     (32, 5, 2, 128),
-    (33, 4, 2, 128),
+    (33, 4, 2, 128),       # 48-row boxes, three m-tiles
+    (40, 3, 2, 64),
+    (48, 3, 1, 128),
     (64, 3, 1, 32),
     (65, 3, 2, 128),       # long clip: tensor-core kernel over a strided view
     (150, 2, 1, 128),
