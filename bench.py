@@ -441,7 +441,7 @@ def main():
     full_ms = per_row["attn_full"]
     achieved = full_f / (full_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
-    roofline = {"bound": "tensor", "kernel": "attn_fwd_tcgen05_kernel<128>", "achieved": achieved, "peak": peak,
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_tcgen05_kernel<128, false>", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": stored_traffic(args.workload),
                 "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside a long step)",
                 "frac_of_burst": achieved / peaks["bf16_tflops"],

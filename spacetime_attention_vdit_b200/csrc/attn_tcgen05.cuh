@@ -145,10 +145,11 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_
   }
 }
 
-template <int D>
+template <int D, bool kStageO>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                            const AttnParams p) {
   using C = AttnCfg<D>;
   unsigned char* smem_raw = dyn_smem;
   const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
@@ -383,24 +384,64 @@ __global__ void __launch_bounds__(320, 1)
     }
 
     // ------------------------------------------------------------- epilogue
-    if (ok && warp_wait(drain, 0, kSiteODone)) {
-      tc_fence_after();
-      const int i = q0 + tile * C::BM + row;      // position in the sequence
-      const float inv_l = 1.f / l_sum;
-      long long token;
-      if (p.mode == kTime) {
-        const int b = bb / p.grp, sidx = bb % p.grp;
-        token = (long long)b * p.L * p.grp + (long long)i * p.grp + sidx;
-      } else {
-        token = (long long)bb * p.L + i;
-      }
-      __nv_bfloat16* orow = p.o + (token * p.heads + h) * D;
+    if constexpr (!kStageO) {
+      // each thread writes its own row of O with 16-byte stores
+      if (ok && warp_wait(drain, 0, kSiteODone)) {
+        tc_fence_after();
+        const int i = q0 + tile * C::BM + row;      // position in the sequence
+        const float inv_l = 1.f / l_sum;
+        long long token;
+        if (p.mode == kTime) {
+          const int b = bb / p.grp, sidx = bb % p.grp;
+          token = (long long)b * p.L * p.grp + (long long)i * p.grp + sidx;
+        } else {
+          token = (long long)bb * p.L + i;
+        }
+        __nv_bfloat16* orow = p.o + (token * p.heads + h) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(t_o + c * 32, o);
-        tmem_ld_wait();
-        if (i < p.L) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait();
+          if (i < p.L) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+              v.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+              v.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+              v.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+            }
+          }
+        }
+        if (p.lse != nullptr && i < p.L) {
+          const int b = bb / p.grp, g = bb % p.grp;
+          const long long pos = p.mode == kTime ? (long long)i * p.grp + g : (long long)g * p.L + i;
+          p.lse[((long long)b * p.heads + h) * ((long long)p.L * p.grp) + pos] =
+              (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+        }
+      }
+    } else {
+      // O / l is staged in this tile's Q buffer (every UMMA, the QK^T ones that
+      // read Q included, has finished once `drain` fires) in the layout of the
+      // Q tensor map; then one thread sends the tile with one TMA store per
+      // D-block, rows past the sequence end clipped, so whole 128-byte lines
+      // leave the SM instead of a 16-byte piece per row and lane
+      bool good = ok;
+      if (good) good = warp_wait(drain, 0, kSiteODone);
+      if (good) {
+        tc_fence_after();
+        const int i = q0 + tile * C::BM + row;      // position in the sequence
+        const float inv_l = 1.f / l_sum;
+        unsigned char* stage = sQ + tile * C::TILE_BYTES;
+        const int key = C::ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
+        constexpr int CPB = C::ROWB / 16;           // 16-byte chunks per staged row
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
@@ -408,15 +449,29 @@ __global__ void __launch_bounds__(320, 1)
             v.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
             v.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
             v.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+            const int cc = c * 4 + e / 8;           // 16-byte chunk of the row
+            *reinterpret_cast<uint4*>(stage + (cc / CPB) * C::DB_BYTES + row * C::ROWB +
+                                      (((cc % CPB) ^ key) << 4)) = v;
           }
         }
+        if (p.lse != nullptr && i < p.L) {
+          const int b = bb / p.grp, g = bb % p.grp;
+          const long long pos = p.mode == kTime ? (long long)i * p.grp + g : (long long)g * p.L + i;
+          p.lse[((long long)b * p.heads + h) * ((long long)p.L * p.grp) + pos] =
+              (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+        }
       }
-      if (p.lse != nullptr && i < p.L) {
-        const int b = bb / p.grp, g = bb % p.grp;
-        const long long pos = p.mode == kTime ? (long long)i * p.grp + g : (long long)g * p.L + i;
-        p.lse[((long long)b * p.heads + h) * ((long long)p.L * p.grp) + pos] =
-            (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+      // the staged rows become visible to the TMA engine; the tile's four
+      // warps meet, and the store goes out only if all four staged their rows
+      fence_proxy_async_smem();
+      const bool all_good = named_bar_and(1 + tile, 128, good);
+      if (all_good && quad == 0 && lane == 0) {
+#pragma unroll
+        for (int db = 0; db < C::NDB; ++db)
+          tma_store_5d(&tmO, sQ + tile * C::TILE_BYTES + db * C::DB_BYTES, db * C::DBLK, h, c_site,
+                       q0 + tile * C::BM, c_batch);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();                  // the buffer is read before the CTA exits
       }
     }
   }

@@ -109,15 +109,20 @@ bool make_2d_map(CUtensorMap* map, const void* base, long long cols, long long r
 // Attention launches
 // ---------------------------------------------------------------------------
 
+// Key tiles (of 128 keys) up to which the kernel stages O for TMA stores.
+constexpr int kStagedOMaxKeyTiles = 16;
+
 template <int D>
 int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq, int L,
                    int Lk, int grp, int heads, float scale, cudaStream_t stream) {
   using C = AttnCfg<D>;
-  static bool smem_done[kMaxDevices] = {};
+  static bool smem_row[kMaxDevices] = {}, smem_staged[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (!ensure_smem(attn_fwd_tcgen05_kernel<D>, C::SMEM_BYTES, smem_done)) return VDIT_ERR_CUDA;
+    if (!ensure_smem(attn_fwd_tcgen05_kernel<D, false>, C::SMEM_BYTES, smem_row) ||
+        !ensure_smem(attn_fwd_tcgen05_kernel<D, true>, C::SMEM_BYTES, smem_staged))
+      return VDIT_ERR_CUDA;
   }
   // geometry of the 5-D view
   long long sites, positions, batches, site_stride, pos_stride, batch_stride;
@@ -141,10 +146,12 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
   // come from another token array (cross-attention; kSeq only)
   const long long k_positions = mode == kTime ? positions : Lk;
   const long long k_batch_stride = mode == kTime ? batch_stride : tok * Lk;
-  CUtensorMap mq, mk, mv;
+  // O is written through a map of the same shape as Q's (the kernel's TMA stores)
+  CUtensorMap mq, mk, mv, mo;
   if (!make_qkv_map(&mq, q, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride) ||
       !make_qkv_map(&mk, k, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride) ||
-      !make_qkv_map(&mv, v, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride))
+      !make_qkv_map(&mv, v, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride) ||
+      !make_qkv_map(&mo, o, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride))
     return VDIT_ERR_CUDA;
   AttnParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -160,7 +167,14 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = (long long)n_seq * heads * p.n_qblocks;
   if (grid > 0x7fffffffLL) return VDIT_ERR_SHAPE;
-  attn_fwd_tcgen05_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  // Short key sequences (cross-attention to a prompt, the space pass at 480p)
+  // give each CTA few key tiles, so its epilogue weighs: O goes out staged in
+  // shared memory by TMA stores.  Long ones keep the per-row stores, whose
+  // variant of the kernel runs its key-tile loop faster.
+  if (p.n_kv <= kStagedOMaxKeyTiles)
+    attn_fwd_tcgen05_kernel<D, true><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  else
+    attn_fwd_tcgen05_kernel<D, false><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
   return last_launch_status();
 }
 
