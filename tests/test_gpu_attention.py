@@ -84,6 +84,8 @@ def test_tiny_divided_equals_masked_full():
     (2, 200, 2, 32),
     (1, 300, 1, 128),
     (1, 1000, 2, 128),     # several tiles and a ragged tail
+    (1, 2048, 1, 128),     # 16 key tiles: the last length whose O is staged for TMA stores
+    (1, 2100, 1, 64),      # 17 key tiles: per-row stores
 ])
 def test_full_ragged(B, L, H, D):
     import spacetime_attention_vdit_b200 as v_

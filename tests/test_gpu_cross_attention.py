@@ -41,6 +41,7 @@ def cross_inputs(B, Lq, Lk, H, D, seed, q_scale=1.0):
     (2, 1000, 512, 3, 128, 1.0),  # 512 prompt tokens, several query blocks
     (1, 500, 512, 2, 128, 8.0),   # peaked rows
     (1, 130, 700, 2, 64, 1.0),    # more keys than queries
+    (2, 300, 2200, 2, 128, 1.0),  # 18 key tiles: the per-row-store variant of the kernel
 ])
 def test_cross_small(B, Lq, Lk, H, D, q_scale):
     import spacetime_attention_vdit_b200 as v_
