@@ -30,6 +30,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -82,13 +83,21 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def code_only(src):
+    """C++ source without its comments and blank lines, each line stripped: what
+    the compiler sees, so that editing a comment does not change the hash."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).strip() for ln in src.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash():
-    """Hash of the attention kernel's sources: a stored ncu traffic figure is used
-    only while it still describes the kernel that runs."""
+    """Hash of the attention kernel's code (comments excluded): a stored ncu
+    traffic figure is used only while it still describes the kernel that runs."""
     h = hashlib.sha256()
     for f in ("attn_tcgen05.cuh", "ptx.cuh"):
-        with open(os.path.join(ROOT, "spacetime_attention_vdit_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "spacetime_attention_vdit_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

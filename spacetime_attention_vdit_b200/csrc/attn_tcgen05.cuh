@@ -28,6 +28,10 @@
 // P = 2^(s * scale * log2e - m) rounded to bf16, one pair in kFmaPairEvery
 // exponentiated on the FMA pipe to unload the MUFU; O rescaled in TMEM only
 // when m moved; at the end O / l and the row's log-sum-exp are written out.
+// kStageO picks how O leaves the SM: false, each thread stores its own row
+// with 16-byte stores; true, the rows are staged in the tile's Q buffer and
+// sent with TMA stores, which pays off when a CTA sweeps only a few key tiles
+// (the host picks true up to 16 key tiles).
 //
 // Each CTA sweeps the key tiles starting at tile (query block mod tiles), so
 // the CTAs of one head, which run together, read different K/V lines from L2
