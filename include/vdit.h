@@ -262,6 +262,21 @@ const char* vdit_status_string(int status);
  */
 int vdit_device_status(unsigned int* flags);
 
+/*
+ * vdit_watchdog_selftest - exercise the failure-detection path.  Enqueues on
+ * `stream` one kernel whose single bounded wait (on an mbarrier that nothing
+ * arrives on) runs out after the 2-second limit every wait in the library has,
+ * and records `site` (1..255) in the device flags exactly as a stalled
+ * pipeline would.  Nothing faults and the context stays usable: a following
+ * vdit_device_status() returns VDIT_ERR_TIMEOUT with flags bit 0 set and
+ * `site` in bits 8..15, and clears them.  While the flag is set, the
+ * library's kernels give up at their first wait that does not complete at
+ * once (the simplest ones do not start), so their results are not valid: call
+ * vdit_device_status() before further work.  Errors: VDIT_ERR_SHAPE (site out
+ * of range), VDIT_ERR_CUDA (launch failed).
+ */
+int vdit_watchdog_selftest(int site, vdit_stream_t stream);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int vdit_version(void);
 

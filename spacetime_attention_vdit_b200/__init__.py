@@ -29,7 +29,7 @@ import torch
 
 __all__ = ["VditError", "lib", "patchify_3d", "patch_embed_3d", "unpatchify_3d", "rope_3d",
            "qk_norm_rope_3d", "attn_full", "attn_divided_time", "attn_divided_space", "attn_cross",
-           "device_status", "status_string", "default_split", "LIB_PATH"]
+           "device_status", "watchdog_selftest", "status_string", "default_split", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
 
@@ -60,6 +60,7 @@ _SIGNATURES = {
     "vdit_attn_divided_space": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_cross": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P],
     "vdit_device_status": [ctypes.POINTER(ctypes.c_uint)],
+    "vdit_watchdog_selftest": [_I, _P],
     "vdit_version": [],
 }
 
@@ -315,3 +316,13 @@ def device_status():
     flags = ctypes.c_uint(0)
     rc = lib().vdit_device_status(ctypes.byref(flags))
     return rc, flags.value
+
+
+def watchdog_selftest(site: int = 99) -> None:
+    """Enqueue the library's failure-detection self-check on the current CUDA
+    stream: a kernel whose one bounded wait can never complete runs out after
+    the 2-second limit and records ``site`` in the device flags, which the next
+    :func:`device_status` reports (VDIT_ERR_TIMEOUT) and clears."""
+    rc = lib().vdit_watchdog_selftest(int(site), _stream(None))
+    if rc != 0:
+        raise VditError("vdit_watchdog_selftest", rc)

@@ -225,6 +225,19 @@ int dispatch_time_short_tp(const void* q, const void* k, const void* v, const Ti
 
 float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)D); }
 
+// Self-check of the bounded wait: one thread waits on an mbarrier that nothing
+// will ever arrive on, so the wait runs out after kWaitLimitNs (or at once if
+// the flag is already set) and records `site`, exactly as a stalled pipeline
+// inside one of the library's kernels would.  Nothing faults and nothing is
+// left in flight; the host reads the flag with vdit_device_status.
+__global__ void watchdog_selftest_kernel(int site) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, site);
+}
+
 int check_attn_args(const void* q, const void* k, const void* v, const void* o, const float* lse, long long B,
                     long long L, int heads, int D) {
   if (!q || !k || !v || !o) return VDIT_ERR_NULL;
@@ -255,6 +268,12 @@ const char* vdit_status_string(int status) {
     case VDIT_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     default: return "unknown status";
   }
+}
+
+int vdit_watchdog_selftest(int site, vdit_stream_t stream) {
+  if (site < 1 || site > 255) return VDIT_ERR_SHAPE;
+  watchdog_selftest_kernel<<<1, 32, 0, stream>>>(site);
+  return last_launch_status();
 }
 
 int vdit_device_status(unsigned int* flags) {

@@ -119,6 +119,12 @@ def test_attention_validation(L, fn, dims):
     assert attn(L, fn, dims=neg) == SHAPE
 
 
+def test_watchdog_selftest_site_checked(L):
+    assert L.vdit_watchdog_selftest(0, None) == SHAPE
+    assert L.vdit_watchdog_selftest(256, None) == SHAPE
+    assert L.vdit_watchdog_selftest(-1, None) == SHAPE
+
+
 def test_cross_key_length_checked(L):
     assert attn(L, "vdit_attn_cross", dims=(1, 256, 0, 2, 128)) == SHAPE
     assert attn(L, "vdit_attn_cross", dims=(1, 256, -3, 2, 128)) == SHAPE
@@ -190,7 +196,7 @@ def test_register_budget_fits_each_sm_subpartition():
             regs[name] = int(m.group(1))
     threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256,
                "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256, "patch_embed_kernel": 320,
-               "unpatchify3d_kernel": 256}
+               "unpatchify3d_kernel": 256, "watchdog_selftest_kernel": 32}
 
     def block_of(kname):
         for key, t in threads.items():
