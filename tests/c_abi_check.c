@@ -60,5 +60,6 @@ int main(void) {
   expect("cross lse align",
          vdit_attn_cross(fake, fake, fake, fake, (float*)((char*)fake + 2), 1, 256, 77, 2, 128, 0.f, NULL),
          VDIT_ERR_ALIGN);
+  expect("watchdog self-test site", vdit_watchdog_selftest(0, NULL), VDIT_ERR_SHAPE);
   return fails;
 }
