@@ -174,8 +174,8 @@ class ClockSampler:
 
 def oracle_sample(d, budget_s, seed=0):
     """Time the float64 oracle on a bounded sample of the step: query rows of full
-    attention of one (batch, head), plus proportional rows of the space pass.
-    Returns (FLOPs done, seconds, description)."""
+    attention of one (batch, head), plus the same rows of the space and time
+    passes.  Returns (FLOPs done, seconds, description, query rows done)."""
     import synthetic
     from oracle import reference as ref
 
@@ -201,7 +201,14 @@ def oracle_sample(d, budget_s, seed=0):
         per_row = el / done_rows
         rows = int(max(16, min(4096, rows * 2, (budget_s - el) / per_row + 1)))
     return flops, el, f"{done_rows} query rows of one (batch, head): full attention over all {L} keys, " \
-                      f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy"
+                      f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy", done_rows
+
+
+def oracle_rates(d, flops, seconds, rows):
+    """Measured oracle rows per second, and the time a whole step would take at the
+    measured FLOP rate (extrapolated: the oracle never runs a whole step)."""
+    return {"rows_per_s": rows / seconds,
+            "extrapolated_step_s": sum(step_flops(d)) / (flops / seconds)}
 
 
 def rank_seed(rank: int) -> int:
@@ -240,11 +247,12 @@ def run_reference(args, d):
     per_step_budget = max(1.0, min(20.0, 150.0 / max(1, steps + warmup)))
     for _ in range(warmup):
         oracle_sample(d, per_step_budget / 4)
-    tot_f, tot_s, desc = 0, 0.0, ""
+    tot_f, tot_s, tot_r, desc = 0, 0.0, 0, ""
     for _ in range(steps):
-        f, s, desc = oracle_sample(d, per_step_budget)
+        f, s, desc, r = oracle_sample(d, per_step_budget)
         tot_f += f
         tot_s += s
+        tot_r += r
     val = tot_f / tot_s / 1e12
     line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * tot_s / steps, "higher_is_better": True,
@@ -252,7 +260,7 @@ def run_reference(args, d):
             "config": {"workload": args.workload, "description": d["desc"], "batch": d["B"], "tokens": d["L"],
                        "heads": d["heads"], "head_dim": d["D"]},
             "cpu_baseline": {"kind": "oracle", "value": val, "unit": "TFLOP/s", "cores": cpu_cores(),
-                             "sample": f"per step: {desc}"},
+                             "sample": f"per step: {desc}", **oracle_rates(d, tot_f, tot_s, tot_r)},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -580,9 +588,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, s, desc = oracle_sample(d, 15.0)
+        f, s, desc, r = oracle_sample(d, 15.0)
         cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": desc + f"; {s:.1f} s"}
+               "sample": desc + f"; {s:.1f} s", **oracle_rates(d, f, s, r)}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
