@@ -213,7 +213,7 @@ int launch_time_short(const void* q, const void* k, const void* v, const TimePar
 }
 
 template <int D>
-int dispatch_time_short_tp(const void* q, const void* k, const void* v, const TimeParams& p,
+int dispatch_time_short(const void* q, const void* k, const void* v, const TimeParams& p,
                            cudaStream_t stream) {
   // box rows: T rounded up to 8 (16 at least), from the set compiled here
   if (p.T <= 16) return launch_time_short<D, 16>(q, k, v, p, stream);
@@ -546,9 +546,9 @@ int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o,
   p.B = B; p.T = T; p.HW = HW; p.heads = heads;
   p.scale_log2 = sc * 1.4426950408889634f;
   switch (head_dim) {
-    case 32: return dispatch_time_short_tp<32>(q, k, v, p, st);
-    case 64: return dispatch_time_short_tp<64>(q, k, v, p, st);
-    case 128: return dispatch_time_short_tp<128>(q, k, v, p, st);
+    case 32: return dispatch_time_short<32>(q, k, v, p, st);
+    case 64: return dispatch_time_short<64>(q, k, v, p, st);
+    case 128: return dispatch_time_short<128>(q, k, v, p, st);
     default: return VDIT_ERR_UNSUPPORTED;
   }
 }
