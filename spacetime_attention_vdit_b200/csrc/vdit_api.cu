@@ -1,9 +1,9 @@
 // vdit_api.cu - the C ABI of libvdit.so (declared in include/vdit.h).
 //
-// Host side only: argument checks that return before any launch, tensor-map
-// encoding for the TMA loads, grid sizing, and the launches themselves.  One
-// translation unit holds every kernel so that the watchdog flag is a single
-// device symbol.
+// Host side, apart from the watchdog's self-check kernel: argument checks that
+// return before any launch, tensor-map encoding for the TMA loads and stores,
+// grid sizing, and the launches themselves.  One translation unit holds every
+// kernel so that the watchdog flag is a single device symbol.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
