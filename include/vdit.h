@@ -58,9 +58,19 @@
  *    unsupported head_dim) return before anything is launched.  A failed
  *    launch returns VDIT_ERR_CUDA.  Faults during execution surface on the
  *    caller's stream, as for any CUDA kernel.
- *  - Every wait inside a kernel is bounded.  A wait that runs out records a
- *    flag that vdit_device_status() reports (VDIT_ERR_TIMEOUT); until the flag
- *    is cleared, later launches exit at once instead of computing.
+ *  - Failure detection.  Every wait inside a kernel is bounded (2 s).  A wait
+ *    that runs out sets a flag word that is ONE per device: every call, stream
+ *    and host thread using the device shares it.  While it is set, every later
+ *    launch of this library on that device, on any stream, produces no valid
+ *    output: the gather and rotation kernels return without writing, and the
+ *    tensor-core kernels give up at the first wait that does not complete
+ *    within its first 64 polls.  Those calls still return VDIT_OK, because the
+ *    host cannot see a device flag without synchronising.  Only
+ *    vdit_device_status() reads the flag: it synchronises the whole device,
+ *    returns VDIT_ERR_TIMEOUT with the site of the first wait that ran out, and
+ *    clears the flag.  A caller that must know that a particular call's output
+ *    is valid calls vdit_device_status() after it.  Each call below notes this
+ *    as "Watchdog: device-wide".
  */
 #ifndef VDIT_H
 #define VDIT_H
@@ -102,6 +112,7 @@ enum vdit_dtype { VDIT_F32 = 0, VDIT_BF16 = 1 };
  * 16-byte alignment enables vector access.  Errors: VDIT_ERR_NULL,
  * VDIT_ERR_SHAPE (a non-positive size, a grid extent of 0, or more than 2^31
  * tokens), VDIT_ERR_UNSUPPORTED (dtype), VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
                      int N, int C, int T, int H, int W,
@@ -127,6 +138,7 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
  * negative part - the page's rope_3d ValueError; non-positive sizes),
  * VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED (head_dim not a multiple of 8),
  * VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
                  int B, int Tg, int Hg, int Wg, int heads, int head_dim,
@@ -147,6 +159,7 @@ int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
  * accumulation, rounded once.  Extents that do not divide are floored.
  * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED
  * (C*pt*ph*pw other than 64, or dim not a multiple of 256), VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bias, void* out,
                         int N, int C, int T, int H, int W, int pt, int ph, int pw, int dim,
@@ -160,6 +173,7 @@ int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bi
  * must not overlap.
  * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_UNSUPPORTED (dtype, or a token
  * wider than 32 KB), VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C, int Tg, int Hg, int Wg,
                        int pt, int ph, int pw, vdit_stream_t stream);
@@ -182,6 +196,7 @@ int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C
  * whole token whose 16-byte vectors, norm_group/8, do not divide 32;
  * heads*head_dim above 8,192; Tg*d_t/2 + Hg*d_h/2 + Wg*d_w/2 above 8,192),
  * VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
                          const float* wq, const float* wk, int norm_group, float eps,
@@ -200,6 +215,7 @@ int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* 
  * before the P.V product; O is rounded to bfloat16 (nearest even).
  * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE, VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED,
  * VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int L, int heads, int head_dim, float scale,
@@ -215,6 +231,7 @@ int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* 
  * site.  Buffers as for vdit_attn_full (read and written in place of the
  * tokens; nothing is transposed).  lse: NULL or [B, heads, T*HW].
  * Errors as for vdit_attn_full.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int T, int HW, int heads, int head_dim, float scale,
@@ -227,6 +244,7 @@ int vdit_attn_divided_time(const void* q, const void* k, const void* v, void* o,
  * frame t, positions [t*HW, (t+1)*HW); it equals full attention restricted to
  * pairs in the same frame.  Buffers and errors as for
  * vdit_attn_divided_time; lse: NULL or [B, heads, T*HW].
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int T, int HW, int heads, int head_dim, float scale,
@@ -244,6 +262,7 @@ int vdit_attn_divided_space(const void* q, const void* k, const void* v, void* o
  * q, o: [B, Lq, heads, head_dim]; k, v: [B, Lk, heads, head_dim]; lse: NULL or
  * [B, heads, Lq].  No positions are applied (text tokens carry none).
  * Numerics, alignment and errors as for vdit_attn_full.
+ * Watchdog: device-wide (see the conventions above).
  */
 int vdit_attn_cross(const void* q, const void* k, const void* v, void* o, float* lse,
                     int B, int Lq, int Lk, int heads, int head_dim, float scale,

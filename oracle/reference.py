@@ -82,13 +82,18 @@ def unpatchify(tokens: np.ndarray, C: int, grid, pt: int, ph: int, pw: int) -> n
     return np.ascontiguousarray(x.reshape(N, C, Tg * pt, Hg * ph, Wg * pw))
 
 
-def patch_embed(latent: np.ndarray, weight: np.ndarray, bias, pt: int, ph: int, pw: int) -> np.ndarray:
+def patch_embed(latent: np.ndarray, weight: np.ndarray, bias, pt: int, ph: int, pw: int,
+                tokens=None) -> np.ndarray:
     """The patch embedding: a Conv3d whose stride equals its kernel (cheatsheet
     "Tiny video DiT"; towardsai section 4: each 1x2x2 brick of 16 latent channels
     becomes one model-width token), i.e. patchify then a matrix product, in
     float64.  ``weight`` is the Conv3d weight [dim, C, pt, ph, pw] flattened to
-    [dim, C*pt*ph*pw]; ``bias`` is [dim] or None.  Returns [N, L, dim]."""
+    [dim, C*pt*ph*pw]; ``bias`` is [dim] or None.  ``tokens`` optionally keeps
+    only those token rows (each row is its own product, so a subset is exactly
+    those rows of the full result).  Returns [N, L or len(tokens), dim]."""
     tok = patchify(np.asarray(latent, dtype=np.float64), pt, ph, pw)
+    if tokens is not None:
+        tok = tok[:, np.asarray(tokens)]
     w = np.asarray(weight, dtype=np.float64)
     y = tok @ w.T
     if bias is not None:

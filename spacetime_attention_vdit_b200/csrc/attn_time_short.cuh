@@ -173,7 +173,9 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
   int j = 0;                                 // this group's problem count
   for (int k = cg; k < n_local; k += C::NP, ++j) {
     const int st = cg * 2 + (j & 1);
-    if (!mbar_wait(&full[st], (j >> 1) & 1, 22)) break;
+    // every lane of the warp leaves together: the loop body is full of
+    // warp-synchronous ldmatrix, mma.sync and shuffles
+    if (!warp_wait(&full[st], (j >> 1) & 1, 22)) break;
     unsigned char* sb = stages + st * C::STAGE_BYTES;
     const uint32_t aQ = smem_u32(sb), aK = aQ + C::TENSOR_BYTES, aV = aQ + 2 * C::TENSOR_BYTES;
     const long long u = u_begin + k;

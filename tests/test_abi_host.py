@@ -173,7 +173,7 @@ def test_build_command_targets_sm100a():
     assert "-lineinfo" in cmd
 
 
-def test_register_budget_fits_each_sm_subpartition():
+def test_register_budget_fits_each_sm_subpartition(tmp_path):
     """Every kernel's registers x the warps one SM sub-partition receives fit its
     16,384 registers (warps of a CTA are spread round-robin over 4 sub-partitions),
     so no launch can fail for lack of registers.  Uses ptxas's own report."""
@@ -182,7 +182,7 @@ def test_register_budget_fits_each_sm_subpartition():
     from spacetime_attention_vdit_b200 import build
     if shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"):
         pytest.skip("nvcc not available")
-    out = "/tmp/vdit_regcheck.so"
+    out = str(tmp_path / "vdit_regcheck.so")
     res = subprocess.run(build.command(ptxas_verbose=True, out=out), capture_output=True, text=True)
     assert res.returncode == 0, res.stderr[-2000:]
     regs = {}

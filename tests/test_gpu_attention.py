@@ -221,21 +221,35 @@ def test_720p_81_frames_sampled():
     _sampled_full(1, (21, 45, 80), 40)
 
 
-def test_720p_divided_sampled():
-    """Divided attention at 720p: time pass (3,600 sites x 21 frames) and space pass
-    (21 frames x 3,600 sites), 40 heads, 4,096 rows per head each."""
+def _sampled_divided(B, T, HW, H, seed=0, rows_per_head=4096):
+    """Both divided passes on [B, T*HW, H, 128] seeded inputs, compared with the
+    oracle on `rows_per_head` seeded rows of every (batch, head)."""
     import spacetime_attention_vdit_b200 as v_
-    T, HW, H = 21, 3600, 40
-    q, k, v = synthetic.qkv_bf16(1, T * HW, H, 128, seed=0)
+    q, k, v = synthetic.qkv_bf16(B, T * HW, H, 128, seed=seed)
     Q, K, V = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
     ot, lt = v_.attn_divided_time(Q, K, V, T, HW, lse=True)
     os_, ls = v_.attn_divided_space(Q, K, V, T, HW, lse=True)
-    rows = synthetic.sample_rows(T * HW, 4096, seed=0)
+    rows = synthetic.sample_rows(T * HW, rows_per_head, seed=seed)
     ot_g, lt_g = from_dev_bf16(ot[:, rows]), lt[:, :, rows].cpu().numpy()
     os_g, ls_g = from_dev_bf16(os_[:, rows]), ls[:, :, rows].cpu().numpy()
+    del Q, K, V, ot, lt, os_, ls
     for h in range(H):
         qh, kh, vh = f64(q[:, :, h:h + 1]), f64(k[:, :, h:h + 1]), f64(v[:, :, h:h + 1])
         eo, el = ref.divided_time_rows(qh, kh, vh, T, HW, rows)
         assert_attention_close(f64(ot_g[:, :, h:h + 1]), eo, lt_g[:, h:h + 1], el, f"time head {h}")
         eo, el = ref.divided_space_rows(qh, kh, vh, T, HW, rows)
         assert_attention_close(f64(os_g[:, :, h:h + 1]), eo, ls_g[:, h:h + 1], el, f"space head {h}")
+
+
+def test_720p_divided_sampled():
+    """Divided attention at 720p: time pass (3,600 sites x 21 frames) and space pass
+    (21 frames x 3,600 sites), 40 heads, 4,096 rows per head each."""
+    _sampled_divided(1, 21, 3600, 40)
+
+
+def test_480p_81_frames_cfg_pair_divided_sampled():
+    """The divided passes at the shape the bench times: batch 2 (CFG pair), 21
+    frames of 1,560 sites (30x52), 40 heads x 128; 4,096 rows per (batch, head).
+    The space pass sweeps 13 key tiles per frame, so it runs the variant that
+    stages O for TMA stores; the time pass uses 24-row boxes."""
+    _sampled_divided(2, 21, 1560, 40)

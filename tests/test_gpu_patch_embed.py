@@ -65,7 +65,7 @@ def _embed_check(N, C, T, H, W, patch, dim, with_bias=True, tokens=None, seed=7)
     lat_r = synthetic.bf16_bits_to_f64(synthetic.f32_to_bf16_bits(lat))     # the operand the kernel uses
     w64 = synthetic.bf16_bits_to_f64(w_bits)
     toks = np.arange(L) if tokens is None else tokens
-    exp = ref.patch_embed(lat_r, w64, None if b is None else b.astype(np.float64), pt, ph, pw)[:, toks]
+    exp = ref.patch_embed(lat_r, w64, None if b is None else b.astype(np.float64), pt, ph, pw, tokens=toks)
     got = synthetic.bf16_bits_to_f64(from_dev_bf16(out)[:, toks])
     brick = np.abs(ref.patchify(lat_r, pt, ph, pw)[:, toks])
     mag_terms = brick @ np.abs(w64).T + (0.0 if b is None else np.abs(b.astype(np.float64)))
@@ -80,6 +80,8 @@ def _embed_check(N, C, T, H, W, patch, dim, with_bias=True, tokens=None, seed=7)
     (1, 16, 3, 10, 14, (1, 2, 2), 512, True),      # 105 tokens: one ragged tile
     (2, 16, 3, 11, 15, (1, 2, 2), 768, False),     # floored extents, no bias
     (1, 8, 6, 10, 12, (2, 2, 2), 256, True),       # another brick with 64 features
+    (1, 16, 3, 20, 22, (1, 2, 2), 1280, True),     # 5 N tiles: work groups of 2, 2 and 1
+    (1, 16, 2, 18, 30, (1, 2, 2), 1792, False),    # 7 N tiles: work groups of 2, 2, 2 and 1
 ])
 def test_patch_embed_small(N, C, T, H, W, patch, dim, bias):
     _embed_check(N, C, T, H, W, patch, dim, bias)
@@ -93,3 +95,10 @@ def test_patch_embed_480p_17_frames():
 def test_patch_embed_480p_81_frames_cfg_pair_sampled():
     """[2, 16, 21, 60, 104] -> 2 x 32,760 tokens of width 1,536 (4,096 seeded tokens checked)."""
     _embed_check(2, 16, 21, 60, 104, (1, 2, 2), 1536, tokens=synthetic.sample_rows(32760, 4096, seed=0))
+
+
+def test_patch_embed_480p_81_frames_cfg_pair_width_5120_sampled():
+    """The bench's shape: [2, 16, 21, 60, 104] -> 2 x 32,760 tokens of the 14B
+    model's width 5,120 (40 heads x 128; aicassindra Step 2), 20 N tiles in four
+    work groups of 5; 4,096 seeded tokens checked."""
+    _embed_check(2, 16, 21, 60, 104, (1, 2, 2), 5120, tokens=synthetic.sample_rows(32760, 4096, seed=0))

@@ -88,3 +88,10 @@ def test_qk_norm_rope_480p_17_frames(group):
 def test_qk_norm_rope_480p_81_frames_cfg_pair_sampled(group):
     """32,760 tokens, 40 heads x 128, batch 2: 4,096 seeded tokens checked."""
     _check(2, (21, 30, 52), 40, 128, (44, 42, 42), group, tokens=synthetic.sample_rows(32760, 4096, seed=0))
+
+
+@pytest.mark.parametrize("group", [128, 5120])
+def test_qk_norm_rope_720p_81_frames_sampled(group):
+    """75,600 tokens (21x45x80), 40 heads x 128, batch 1: 4,096 seeded tokens
+    checked, per head and per token (5,120 channels)."""
+    _check(1, (21, 45, 80), 40, 128, (44, 42, 42), group, tokens=synthetic.sample_rows(75600, 4096, seed=0))

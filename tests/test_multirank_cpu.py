@@ -42,3 +42,30 @@ def test_two_gloo_ranks():
     import bench
     # two ranks, 1e12 FLOPs per rank-step, 4 steps in 150 ms -> 53.3 TFLOP/s for the job
     assert abs(bench.job_throughput(2, 1e12, 4, 150.0) - 2 * 4 / 0.150) < 1e-9
+
+
+def test_bench_gpus_flag_starts_the_ranks():
+    """`bench.py --gpus 2` outside torchrun starts two local ranks itself
+    (torch.distributed.run on 127.0.0.1); each joins the group and rank 0
+    reports that it saw both.  Host-only: gloo, no GPU, nothing timed."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--launcher-check"],
+                         cwd=root, env=env, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    assert json.loads(lines[0]) == {"launcher_check": True, "world": 2, "ranks_seen": 2}
+
+
+def test_bench_refuses_a_world_size_other_than_gpus(monkeypatch):
+    import pytest
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "3")
+    with pytest.raises(SystemExit):
+        bench.check_world(2)
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.check_world(2) == 2

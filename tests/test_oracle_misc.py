@@ -143,3 +143,22 @@ def test_rope_token_subset():
     x32 = x.astype(np.float32)
     assert np.array_equal(ref.rope_3d_fp32(x32[:, toks], grid, split, tokens=toks),
                           ref.rope_3d_fp32(x32, grid, split)[:, toks])
+
+
+def test_patch_embed_token_subset_is_those_rows_of_torch_conv3d():
+    """The oracle's token selection (used at full size, where only sampled tokens
+    are checked) returns exactly those rows of torch's float64 conv3d."""
+    import torch
+    from oracle import reference as ref
+    g = np.random.default_rng(54)
+    N, C, T, H, W, dim = 2, 4, 3, 6, 8, 24
+    x = g.standard_normal((N, C, T, H, W))
+    w = g.standard_normal((dim, C * 4))
+    b = g.standard_normal(dim)
+    sel = np.array([0, 5, 17, 35])
+    got = ref.patch_embed(x, w, b, 1, 2, 2, tokens=sel)
+    y = torch.nn.functional.conv3d(torch.from_numpy(x), torch.from_numpy(w.reshape(dim, C, 1, 2, 2)),
+                                   torch.from_numpy(b), stride=(1, 2, 2)).numpy()
+    exp = y.reshape(N, dim, -1).transpose(0, 2, 1)[:, sel]
+    assert got.shape == (N, sel.size, dim)
+    assert np.allclose(got, exp, atol=1e-12)
