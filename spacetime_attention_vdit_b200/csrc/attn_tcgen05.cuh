@@ -9,16 +9,21 @@
 // space pass of divided attention (each frame is a contiguous sequence) and,
 // through a strided tensor map, a time pass with long sequences.
 //
-// One CTA computes two 128-row query tiles (256 rows) of one (sequence, head):
-//   warp 0      TMA producer: Q tiles once; K_j into a K ring and V_j into a
+// One CTA computes two 128-row query tiles (256 rows) of one (sequence, head)
+// with three warpgroups:
+//   warps 0..3  softmax of query tile 0, warps 4..7 of tile 1, one query row
+//               per thread (TMEM lane = row);
+//   warp 8      TMA producer: Q tiles once; K_j into a K ring and V_j into a
 //               V ring (K is needed one P.V product earlier than V);
-//   warp 1      allocates all 512 TMEM columns and issues every UMMA from one
+//   warp 9      allocates all 512 TMEM columns and issues every UMMA from one
 //               thread, in a fixed order: O_i += P_i V_j with P_i read from
 //               TMEM (the softmax overwrote tile i's scores with bf16
 //               probabilities), then at once S_i = Q_i K_{j+1}^T (smem x smem)
 //               into the same columns, for tile 0 and then tile 1;
-//   warps 2..5  softmax of query tile 0, warps 6..9 of tile 1, one query row
-//               per thread (TMEM lane = row).
+//   warps 10,11 idle.
+// The control warpgroup (8..11) gives registers back after set-up and the
+// softmax warpgroups take them (setmaxnreg), so that a softmax thread holds its
+// whole row of 128 scores and its packed probabilities without spilling.
 // The two tiles ping-pong: while one warpgroup exponentiates its scores the
 // tensor core runs the other tile's products.  TMEM columns: S/P of tile i at
 // [128 i, 128 i + 128), O of tile i at [256 + 128 i, ...).
@@ -60,7 +65,12 @@ struct AttnCfg {
   static constexpr int NV = D >= 128 ? 2 : (D >= 64 ? 3 : 4);  // V ring stages
   static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NQ + 1;
   static constexpr int SMEM_BYTES = 1024 + (NQ + NK + NV) * TILE_BYTES + NBARS * 8 + 16;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;                          // three warpgroups
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
+  // registers per thread: at launch (what __launch_bounds__(384, 1) allows),
+  // then per warpgroup after the split
+  static constexpr int REGS_LAUNCH = 168, REGS_SOFTMAX = 216, REGS_CONTROL = 56;
+  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_CONTROL <= THREADS * REGS_LAUNCH, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;                         // tile i: scores / P at 128 i
   static constexpr uint32_t O_COL = 256;                       // tile i: accumulator at 256 + 128 i
@@ -125,32 +135,51 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
 
 // One score pair in kFmaPairEvery is exponentiated on the FMA pipe (ex2_fma2),
 // the rest on the MUFU: the MUFU alone needs about as many cycles per key tile
-// as the tensor core, so a small share moved off it shortens the softmax.
-constexpr int kFmaPairEvery = 32;
+// as the tensor core, so a share moved off it shortens the softmax.
+#ifndef VDIT_FMA_PAIR_EVERY
+#define VDIT_FMA_PAIR_EVERY 32
+#endif
+constexpr int kFmaPairEvery = VDIT_FMA_PAIR_EVERY;
+static_assert(64 % kFmaPairEvery == 0, "pairs per row");
+
+// Packed P columns written per TMEM store (2 keys each).
+#ifndef VDIT_P_STORE_COLS
+#define VDIT_P_STORE_COLS 8
+#endif
+constexpr int kPStoreCols = VDIT_P_STORE_COLS;
+static_assert(kPStoreCols == 8 || kPStoreCols == 16 || kPStoreCols == 32, "TMEM store width");
 
 // P = 2^(s * scale_log2 - m) for one row's 128 scores, packed to bf16 pairs and
-// stored over the row's score columns, 16 keys (8 columns) per store so that
-// few packed values are live at once; the packed partial sums go to sp.
+// stored over the row's score columns (pair i of keys 2i, 2i+1 at column i),
+// kPStoreCols columns per store so that few packed values are live at once;
+// the packed partial sums go to sp.
 __device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_s, float2 sc2, float2 nm2,
                                          float2 (&sp)[4]) {
+  constexpr int G = kPStoreCols;
 #pragma unroll
-  for (int h8 = 0; h8 < 8; ++h8) {
-    uint32_t pk[8];
+  for (int g = 0; g < 64 / G; ++g) {
+    uint32_t pk[G];
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {
-      const int c = h8 >> 1, ee = (h8 & 1) * 16 + e;
+    for (int u = 0; u < G; ++u) {
+      const int pi = g * G + u;                   // pair of the row
+      const int c = pi >> 4, ee = (pi & 15) * 2;
       const float2 x = ffma2(make_float2(__uint_as_float(s[c][ee]), __uint_as_float(s[c][ee + 1])), sc2, nm2);
-      const bool on_fma = ((h8 * 8 + (e >> 1)) % kFmaPairEvery) == kFmaPairEvery - 1;
+      const bool on_fma = (pi % kFmaPairEvery) == kFmaPairEvery - 1;
       const float2 pr = on_fma ? ex2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-      sp[(e >> 1) & 3] = fadd2(sp[(e >> 1) & 3], pr);
-      pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
+      sp[u & 3] = fadd2(sp[u & 3], pr);
+      pk[u] = pack_bf16x2(pr.x, pr.y);
     }
-    tmem_st8(t_s + h8 * 8, pk);
+    if constexpr (G == 8)
+      tmem_st8(t_s + g * G, reinterpret_cast<const uint32_t(&)[8]>(pk));
+    else if constexpr (G == 16)
+      tmem_st16(t_s + g * G, reinterpret_cast<const uint32_t(&)[16]>(pk));
+    else
+      tmem_st32(t_s + g * G, reinterpret_cast<const uint32_t(&)[32]>(pk));
   }
 }
 
 template <int D, bool kStageO>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                             const AttnParams p) {
@@ -197,7 +226,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(drain, 1);
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -206,7 +235,11 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  // Each warpgroup's branch starts with its register budget, so that the code
+  // of each role is compiled for the registers that role holds.
+  if (warp >= 8) {
+  regs_decrease<C::REGS_CONTROL>();
+  if (warp == C::TMA_WARP) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -254,7 +287,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = v_issued - C::NV < 0 ? 0 : v_issued - C::NV; j < v_issued; ++j)
         mbar_drain(&v_full[j % C::NV], (j / C::NV) & 1);
     }
-  } else if (warp == 1) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
@@ -319,9 +352,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_drain(drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    regs_increase<C::REGS_SOFTMAX>();
     // -------------------------------------------------------------- softmax
-    const int tile = (warp - 2) >> 2;             // warps 2..5 -> tile 0, 6..9 -> tile 1
+    const int tile = warp >> 2;                   // warps 0..3 -> tile 0, 4..7 -> tile 1
     const int quad = warp & 3;                    // TMEM lanes this warp may touch
     const int row = quad * 32 + lane;             // query row within the tile
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
@@ -337,6 +372,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, s[c]);
       tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_fence(s[c]);
 
       const int valid = p.Lk - ((j + j0) % n) * C::BN;  // keys of this tile inside the sequence
       if (valid < C::BN) {
@@ -376,6 +413,7 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t o[32];
           tmem_ld32(t_o + c * 32, o);
           tmem_ld_wait();
+          tmem_ld_fence(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(t_o + c * 32, o);
@@ -407,6 +445,7 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t o[32];
           tmem_ld32(t_o + c * 32, o);
           tmem_ld_wait();
+          tmem_ld_fence(o);
           if (i < p.L) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
@@ -446,6 +485,7 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t o[32];
           tmem_ld32(t_o + c * 32, o);
           tmem_ld_wait();
+          tmem_ld_fence(o);
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
@@ -482,7 +522,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(kEmbThreads, 1)
             uint32_t o[32];
             tmem_ld32(tl + ac * kEmbBN + bx * kEmbOutBox + h * 32, o);
             tmem_ld_wait();
+            tmem_ld_fence(o);
             const int col = nt * kEmbBN + bx * kEmbOutBox + h * 32;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {

@@ -128,6 +128,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int si
 }
 
 // ---------------------------------------------------------------------------
+// Per-warpgroup register budgets (every warp of a warpgroup executes the same
+// one).  The increase draws on registers that other warpgroups of the CTA
+// released with a decrease; the launch's registers per thread times its threads
+// must cover the sum of the budgets, or the increase waits forever.
+// ---------------------------------------------------------------------------
+
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register budget");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register budget");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------
 // Proxy fences
 // ---------------------------------------------------------------------------
 
@@ -278,6 +296,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// After tcgen05.wait::ld: ties later uses of the loaded registers to the wait.
+// The load's outputs look ready to the compiler at the load itself; pure
+// arithmetic on them could otherwise be scheduled between the load and the
+// wait.  No instruction is emitted.
+__device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[32]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
 // 32 lanes x 8 columns of 32-bit from registers.
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
@@ -344,10 +370,14 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, i
 // Small numeric helpers
 // ---------------------------------------------------------------------------
 
-// 2^x on the special-function unit (one instruction; approximate, flushes denormals).
+// 2^x on the special-function unit (one instruction; approximate, flushes
+// denormals).  Not volatile: it is a pure function of x, and the compiler must
+// be free to issue the exponentials of the next group of scores while the
+// previous group's results are still being packed and stored to TMEM (the
+// TMEM stores are volatile, and volatile asm keeps its program order).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 

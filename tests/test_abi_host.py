@@ -194,7 +194,7 @@ def test_register_budget_fits_each_sm_subpartition(tmp_path):
         m = re.search(r"Used (\d+) registers", line)
         if m and name:
             regs[name] = int(m.group(1))
-    threads = {"attn_fwd_tcgen05_kernel": 320, "rope3d_kernel": 256, "patchify3d_kernel": 256,
+    threads = {"attn_fwd_tcgen05_kernel": 384, "rope3d_kernel": 256, "patchify3d_kernel": 256,
                "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256, "patch_embed_kernel": 320,
                "unpatchify3d_kernel": 256, "watchdog_selftest_kernel": 32}
 
@@ -211,7 +211,17 @@ def test_register_budget_fits_each_sm_subpartition(tmp_path):
         assert 1024 + nstage * (stage + 16) <= 232448
         return 32 * (1 + (nstage // 2) * wpu)
     assert regs, "no ptxas report"
+    # the attention kernel splits its launch registers between warpgroups
+    # (setmaxnreg): two softmax warpgroups take 216 each, the control warpgroup
+    # keeps 56, which needs exactly 168 per thread at launch (384 threads)
+    src = open(os.path.join(os.path.dirname(build.__file__), "csrc", "attn_tcgen05.cuh")).read()
+    m = re.search(r"REGS_LAUNCH = (\d+), REGS_SOFTMAX = (\d+), REGS_CONTROL = (\d+)", src)
+    launch, soft, ctrl = (int(x) for x in m.groups())
+    assert 2 * 128 * soft + 128 * ctrl <= 384 * launch
+    assert 32 * (2 * soft + ctrl) <= 16384              # one warp of each warpgroup per sub-partition
     for kname, r in regs.items():
+        if "attn_fwd_tcgen05_kernel" in kname:
+            assert r == launch, (kname, r)
         warps = block_of(kname) // 32
         per_sub = -(-warps // 4)                  # warps on the fullest sub-partition
         alloc = -(-r // 8) * 8                    # registers are granted in multiples of 8
