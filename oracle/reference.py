@@ -147,6 +147,19 @@ def rope_tables(grid, split, theta: float = 10000.0, tokens=None):
     return np.concatenate(parts, axis=1)
 
 
+def rope_axis_phasors(grid, split, theta: float = 10000.0) -> np.ndarray:
+    """The RoPE's unit phasors per axis position, float64 [n, 2] of (cos, sin):
+    the Tg*d_t/2 time entries (frame-major, then pair), then Hg*d_h/2 height
+    entries, then Wg*d_w/2 width entries.  The towardsai snippet builds one
+    frequency table per axis and looks each token's angles up by its t, h and w
+    (section 4); this is that per-axis cache, before the lookup."""
+    parts = []
+    for n, d in zip(grid, split):
+        ang = np.outer(np.arange(n, dtype=np.float64), rope_inv_freq(d, theta))   # [n, d/2]
+        parts.append(np.stack([np.cos(ang), np.sin(ang)], axis=-1).reshape(-1, 2))
+    return np.concatenate(parts, axis=0)
+
+
 def rope_3d(x: np.ndarray, grid, split, theta: float = 10000.0, tokens=None) -> np.ndarray:
     """Rotate Q or K ``[B, L, heads, D]`` in float64.
 

@@ -175,6 +175,68 @@ def pin_rope_brute(rope):
 ROPE_PINS = [pin_rope_onehot, pin_rope_complex, pin_rope_relative, pin_rope_norm_identity,
              pin_rope_brute]
 
+
+# The per-axis phasor cache (towardsai section 4: one frequency table per axis,
+# each token's angles looked up by its t, h and w).
+
+def _phasor_index(grid, split, axis, pos, i):
+    """Row of the per-axis table: time block, then height, then width."""
+    start = sum(grid[a] * (split[a] // 2) for a in range(axis))
+    return start + pos * (split[axis] // 2) + i
+
+
+def pin_phasors_brute(phasors):
+    """Each entry is what the brute-force rotation does to a unit vector on that
+    pair at that position (pure-Python loops, one token at a time)."""
+    grid, split = (3, 4, 5), (12, 10, 10)
+    tab = phasors(grid, split)
+    assert tab.shape == (3 * 6 + 4 * 5 + 5 * 5, 2)
+    off = (0, 12, 22)
+    for axis in range(3):
+        for pos in range(grid[axis]):
+            for i in range(split[axis] // 2):
+                x = [0.0] * 32
+                x[off[axis] + 2 * i] = 1.0
+                where = [0, 0, 0]
+                where[axis] = pos
+                r = brute.rope_vector(x, tuple(where), split)
+                got = tab[_phasor_index(grid, split, axis, pos, i)]
+                assert abs(got[0] - r[off[axis] + 2 * i]) < 1e-14 and abs(got[1] - r[off[axis] + 2 * i + 1]) < 1e-14
+
+
+def pin_phasors_page_counts(phasors):
+    """The 81-frame 480p grid [21, 30, 52] with the pairs per axis the page prints
+    (towardsai section 4: 22 for time, 21 each for height and width, from the
+    golden fixture): 21*22 + 30*21 + 52*21 entries; position 0 of every axis
+    block is the identity phasor (1, 0)."""
+    from tests.conftest import golden
+    page = golden("page_numbers.txt")
+    pairs = [int(page[k][0]) for k in ("rope_pairs_t", "rope_pairs_h", "rope_pairs_w")]
+    grid, split = (21, 30, 52), (44, 42, 42)
+    tab = phasors(grid, split)
+    assert tab.shape == (21 * pairs[0] + 30 * pairs[1] + 52 * pairs[2], 2)
+    for axis in range(3):
+        for i in range(split[axis] // 2):
+            assert tuple(tab[_phasor_index(grid, split, axis, 0, i)]) == (1.0, 0.0)
+
+
+def pin_phasors_group(phasors):
+    """Angles grow linearly with the position: entry(p) = entry(1)^p as complex
+    numbers (torch complex128 powers), and every entry has modulus 1."""
+    grid, split = (6, 7, 9), (44, 42, 42)
+    tab = phasors(grid, split)
+    z = torch.complex(torch.from_numpy(tab[:, 0].copy()), torch.from_numpy(tab[:, 1].copy()))
+    assert torch.allclose(z.abs(), torch.ones_like(z.abs()), atol=1e-14)
+    for axis in range(3):
+        for i in range(split[axis] // 2):
+            z1 = z[_phasor_index(grid, split, axis, 1, i)]
+            for pos in range(grid[axis]):
+                zp = z[_phasor_index(grid, split, axis, pos, i)]
+                assert abs(complex(zp) - complex(z1) ** pos) < 1e-12, (axis, pos, i)
+
+
+PHASOR_PINS = [pin_phasors_brute, pin_phasors_page_counts, pin_phasors_group]
+
 # ----------------------------------------------------------------------------
 # Patch embedding and unpatchify  (cheatsheet "Tiny video DiT": a Conv3d whose
 # stride equals its kernel; towardsai section 4: bricks to model-width tokens)

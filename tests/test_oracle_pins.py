@@ -42,6 +42,11 @@ def test_unpatchify_pins():
         pin(ref.unpatchify)
 
 
+@pytest.mark.parametrize("pin", pins.PHASOR_PINS, ids=lambda p: p.__name__)
+def test_phasor_pins(pin):
+    pin(ref.rope_axis_phasors)
+
+
 def test_divided_pins():
     pins.pin_divided_time(ref.divided_time)
     pins.pin_divided_space(ref.divided_space)
@@ -234,3 +239,28 @@ def test_embed_mistakes_caught(bad):
 
 def test_unpatchify_mistake_caught():
     assert _fails(pins.UNPATCHIFY_PINS, unpatchify_spatial_swapped) == 1
+
+
+def _phasor_variant(grid, split, theta=10000.0, axis_order=(0, 1, 2), swap=False, head_width=None, start=0):
+    parts = []
+    for a in axis_order:
+        n, d = grid[a], split[a]
+        j = np.arange(0, d, 2, dtype=np.float64)
+        f = 1.0 / (theta ** (j / (head_width or d)))
+        ang = np.outer(np.arange(start, start + n, dtype=np.float64), f)
+        c, s_ = np.cos(ang), np.sin(ang)
+        parts.append(np.stack([s_, c] if swap else [c, s_], axis=-1).reshape(-1, 2))
+    return np.concatenate(parts, axis=0)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(axis_order=(1, 0, 2)),      # height block before the time block
+    dict(swap=True),                 # (sin, cos) instead of (cos, sin)
+    dict(head_width=128),            # frequencies from the head width
+    dict(start=1),                   # positions counted from 1
+], ids=["axis-order", "sin-cos", "head-width-freq", "one-based"])
+def test_phasor_mistakes_caught(kw):
+    for pin in pins.PHASOR_PINS:
+        pin(_phasor_variant)
+    bad = lambda g, s: _phasor_variant(g, s, **kw)
+    assert _fails(pins.PHASOR_PINS, bad) >= 1
