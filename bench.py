@@ -345,6 +345,52 @@ def time_launches(fn, reps, stream, flush=None):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def rope_q_row(vd, q, k, v, qr, kr, o, grid, stream, dev, peaks, rounds=3):
+    """Q's 3D rotation in the attention prologue against the two-step path
+    (towardsai section 5, Sub-Layer 1, then attention): rotate K alone, then
+    attention that rotates Q itself, against rotating Q and K in a pass, then
+    attention.  The two are timed in alternation, each pass and attention
+    launch with its own events, so that both see the same clock."""
+    import torch
+    B, L, Hh, D = q.shape
+    table = vd.rope_3d_table(grid, D)
+    flops = 4.0 * B * Hh * L * L * D
+
+    def two(ev):
+        ev[0].record(stream)
+        vd.rope_3d(q, k, grid, q_out=qr, k_out=kr)
+        ev[1].record(stream)
+        vd.attn_full(qr, kr, v, out=o)
+        ev[2].record(stream)
+
+    def one(ev):
+        ev[0].record(stream)
+        vd.rope_3d(None, k, grid, k_out=kr)
+        ev[1].record(stream)
+        vd.attn_full_rope_q(q, kr, v, grid, table, out=o)
+        ev[2].record(stream)
+
+    for fn in (two, one):
+        fn([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    evs = {"two": [], "one": []}
+    for _ in range(rounds):
+        for name, fn in (("two", two), ("one", one)):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            fn(e)
+            evs[name].append(e)
+    torch.cuda.synchronize(dev)
+
+    def mean(name, a, b):
+        return statistics.mean(e[a].elapsed_time(e[b]) for e in evs[name])
+    a_ms = mean("one", 1, 2)
+    return {"two_step_ms": mean("two", 0, 2), "one_step_ms": mean("one", 0, 2),
+            "rope_qk_ms": mean("two", 0, 1), "rope_k_ms": mean("one", 0, 1),
+            "attn_ms": mean("two", 1, 2), "attn_rope_q_ms": a_ms,
+            "attn_rope_q_tflops": flops / (a_ms * 1e-3) / 1e12,
+            "attn_rope_q_frac_of_burst": flops / (a_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "rounds": rounds}
+
+
 def other_workloads(vd, dev, stream, peaks):
     """The pages' other clips, each timed on its own after 3 warm-up launches.
 
@@ -727,6 +773,7 @@ def main():
         cross["qk_norm_rope"] = {"norm_group": width, "ms": nms, "gb_s": nbytes / (nms * 1e-3) / 1e9,
                                  "frac_hbm": nbytes / (nms * 1e-3) / 1e9 / peaks["hbm_gbs"], "bytes": nbytes}
         del qn, kn
+        cross["rope_q_in_attention"] = rope_q_row(vd, q, k, v, qr, kr, o_full, grid, stream, dev, peaks)
         # next row: the patch embedding (patchify and the Conv3d weight on the tensor
         # cores) to the model width heads*D of this workload
         dim = Hh * D

@@ -13,6 +13,9 @@
  *     -> vdit_rope_3d            factorised 3D rotary positions on Q and K
  *        (or vdit_qk_norm_rope_3d: RMSNorm of Q and K, then the same rotation)
  *     -> vdit_attn_full          full 3D self-attention over all T*H'*W' tokens
+ *        (or vdit_attn_full_rope_q: Q normalised and rotated inside the
+ *         attention kernel, K by the pass above alone, with the pairs of
+ *         vdit_rope_3d_table)
  *        or
  *        vdit_attn_divided_time  attention over the T tokens at each spatial site
  *        vdit_attn_divided_space attention over the H'*W' tokens of each frame
@@ -133,7 +136,9 @@ int vdit_patchify_3d(const void* latent, void* tokens, int dtype,
  * float32, as the page's snippet does; the rotation runs in float32 with each
  * product and sum rounded separately, and the result is rounded to bfloat16
  * (nearest even).  V is not rotated.  q_out/k_out may equal q_in/k_in (in
- * place); otherwise the buffers must not overlap.  Errors: VDIT_ERR_NULL,
+ * place); otherwise the buffers must not overlap.  q_in and q_out both NULL:
+ * K alone is rotated (for vdit_attn_full_rope_q, which rotates Q itself).
+ * Errors: VDIT_ERR_NULL (also: one of q_in, q_out NULL but not the other),
  * VDIT_ERR_SHAPE (the split does not add up to head_dim or has an odd or
  * negative part - the page's rope_3d ValueError; non-positive sizes),
  * VDIT_ERR_ALIGN, VDIT_ERR_UNSUPPORTED (head_dim not a multiple of 8),
@@ -189,7 +194,8 @@ int vdit_unpatchify_3d(const void* tokens, void* latent, int dtype, int N, int C
  * then rotated exactly as vdit_rope_3d does (same grid, split and theta),
  * float32 throughout and rounded once to bfloat16 (nearest even).
  * wq, wk: NULL (weight 1) or device float32 [norm_group], 16-byte aligned.
- * Layouts, aliasing and the RoPE arguments as for vdit_rope_3d.
+ * Layouts, aliasing, the K-only form (q_in and q_out NULL) and the RoPE
+ * arguments as for vdit_rope_3d.
  * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE (also: norm_group not dividing
  * heads*head_dim, eps negative or not finite), VDIT_ERR_ALIGN,
  * VDIT_ERR_UNSUPPORTED (norm_group not a multiple of 8; a group other than the
@@ -202,6 +208,32 @@ int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* 
                          const float* wq, const float* wk, int norm_group, float eps,
                          int B, int Tg, int Hg, int Wg, int heads, int head_dim,
                          int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
+
+/*
+ * vdit_rope_3d_table - the 3D RoPE's (cos, sin) pairs for one token grid
+ * [towardsai s.4: the snippet computes its phasors once per shape and keeps
+ * them as a cache].
+ *
+ * table: device float32 [n][2], n = Tg*(d_t/2) + Hg*(d_h/2) + Wg*(d_w/2)
+ * (vdit_rope_3d_table_entries), 16-byte aligned, written by the call:
+ *   entry t'*(d_t/2) + i                          time pair i at frame t'
+ *   entry Tg*(d_t/2) + h'*(d_h/2) + i             height pair i at row h'
+ *   entry Tg*(d_t/2) + Hg*(d_h/2) + w'*(d_w/2) + i  width pair i at column w'
+ * each holding (cos a, sin a) of a = pos * theta^(-2i/d) for its segment width
+ * d, formed in float64 and rounded once to float32: the values vdit_rope_3d
+ * rotates with.  The table depends only on the grid, the split and theta; it
+ * is an input of vdit_attn_full_rope_q and can be reused by every call on that
+ * grid.  Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE (the split or theta as for
+ * vdit_rope_3d; more than 2^31 - 1 entries), VDIT_ERR_ALIGN, VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
+ */
+int vdit_rope_3d_table(float* table, int Tg, int Hg, int Wg, int head_dim,
+                       int d_t, int d_h, int d_w, float theta, vdit_stream_t stream);
+
+/* Entries (float32 pairs) of vdit_rope_3d_table's table, or -1 for a bad grid
+ * or split.  Host only; launches nothing. */
+long long vdit_rope_3d_table_entries(int Tg, int Hg, int Wg, int head_dim,
+                                     int d_t, int d_h, int d_w);
 
 /*
  * vdit_attn_full - full 3D self-attention [towardsai s.5: every token attends
@@ -220,6 +252,37 @@ int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* 
 int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int L, int heads, int head_dim, float scale,
                    vdit_stream_t stream);
+
+/*
+ * vdit_attn_full_rope_q - full 3D self-attention whose kernel normalises and
+ * rotates Q itself [towardsai s.5, "Sub-Layer 1": the projected Q and K are
+ * RMS-normalised, rotated with the 3D RoPE of s.4, then attend to each other].
+ *
+ *   O = vdit_attn_full(q', k, v)   with   q' = rope_3d(norm(q))
+ *
+ * where norm is the identity (norm_group 0) or the per-head RMSNorm of
+ * vdit_qk_norm_rope_3d with norm_group = head_dim and weight wq, and rope_3d
+ * is vdit_rope_3d's rotation with the pairs of `rope_table`
+ * (vdit_rope_3d_table of the same grid, split and theta).  q' is never
+ * written to memory: each CTA rewrites the Q rows it loads, in shared memory,
+ * before its first Q.K^T, with the stand-alone passes' arithmetic, so O is the
+ * same, bit for bit, as that of the two-step path.  k must already be
+ * normalised and rotated (vdit_qk_norm_rope_3d or vdit_rope_3d with q_in and
+ * q_out NULL).  A token-wide norm (norm_group = heads*head_dim) needs every head
+ * of a token, which one attention CTA does not load: run it with
+ * vdit_qk_norm_rope_3d.  q, k, v, o: [B, L, heads, head_dim] with
+ * L = Tg*Hg*Wg; lse, numerics and alignment as for vdit_attn_full; wq: NULL
+ * (weight 1) or device float32 [head_dim], 16-byte aligned.
+ * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE (also: the split as for vdit_rope_3d,
+ * eps negative or not finite when normalising), VDIT_ERR_ALIGN,
+ * VDIT_ERR_UNSUPPORTED (head_dim; norm_group other than 0 or head_dim),
+ * VDIT_ERR_CUDA.
+ * Watchdog: device-wide (see the conventions above).
+ */
+int vdit_attn_full_rope_q(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Tg, int Hg, int Wg, int heads, int head_dim, float scale,
+                          int d_t, int d_h, int d_w, const float* rope_table,
+                          const float* wq, int norm_group, float eps, vdit_stream_t stream);
 
 /*
  * vdit_attn_divided_time - the time pass of divided attention [cheatsheet

@@ -15,7 +15,9 @@ Calls (see ``include/vdit.h`` for the exact definitions and sources):
 * :func:`unpatchify_3d`       tokens [N, L, C*pt*ph*pw] -> latent [N, C, T, H, W]
 * :func:`rope_3d`             3D rotary positions on Q and K [B, L, heads, D]
 * :func:`qk_norm_rope_3d`     RMSNorm of Q and K, then the 3D rotation, in one pass
+* :func:`rope_3d_table`       the 3D RoPE's (cos, sin) pairs per axis position
 * :func:`attn_full`           full 3D self-attention
+* :func:`attn_full_rope_q`    full 3D self-attention that normalises and rotates Q itself
 * :func:`attn_divided_time`   attention over the T tokens of each spatial site
 * :func:`attn_divided_space`  attention over the HW tokens of each frame
 * :func:`attn_cross`          video tokens attending to a separate key/value sequence
@@ -28,7 +30,7 @@ import os
 import torch
 
 __all__ = ["VditError", "lib", "patchify_3d", "patch_embed_3d", "unpatchify_3d", "rope_3d",
-           "qk_norm_rope_3d", "attn_full", "attn_divided_time", "attn_divided_space", "attn_cross",
+           "qk_norm_rope_3d", "rope_3d_table", "attn_full", "attn_full_rope_q", "attn_divided_time", "attn_divided_space", "attn_cross",
            "device_status", "watchdog_selftest", "status_string", "default_split", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdit.so")
@@ -53,6 +55,8 @@ _SIGNATURES = {
     "vdit_patchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_rope_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "vdit_attn_full": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P],
+    "vdit_rope_3d_table": [_P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
+    "vdit_attn_full_rope_q": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P, _P, _I, _F, _P],
     "vdit_patch_embed_3d": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_unpatchify_3d": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P],
     "vdit_qk_norm_rope_3d": [_P, _P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P],
@@ -77,6 +81,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        L.vdit_rope_3d_table_entries.argtypes = [_I] * 7
+        L.vdit_rope_3d_table_entries.restype = ctypes.c_longlong
         L.vdit_status_string.argtypes = [ctypes.c_int]
         L.vdit_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -140,27 +146,60 @@ def patchify_3d(latent: torch.Tensor, patch=(1, 2, 2), out: torch.Tensor | None 
     return out
 
 
-def rope_3d(q: torch.Tensor, k: torch.Tensor, grid, split=None, theta: float = 10000.0,
+def _q_and_out(q, k, q_out, inplace):
+    """Q's input and output pointers; both None when only K is rotated."""
+    if q is None:
+        return None, None, None
+    if q.dim() != 4 or q.shape != k.shape:
+        raise ValueError("q and k must both be [B, L, heads, head_dim]")
+    if inplace:
+        q_out = q
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    return _dev(q, "q", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16), q_out
+
+
+def rope_3d(q: torch.Tensor | None, k: torch.Tensor, grid, split=None, theta: float = 10000.0,
             q_out: torch.Tensor | None = None, k_out: torch.Tensor | None = None, inplace: bool = False,
             stream=None):
     """Rotate Q and K ([B, L, heads, D] bfloat16, L = Tg*Hg*Wg) by their 3D grid
     positions.  ``split`` = (d_t, d_h, d_w), default :func:`default_split`.
-    Returns (q_out, k_out); with ``inplace`` the inputs are overwritten."""
-    if q.dim() != 4 or q.shape != k.shape:
-        raise ValueError("q and k must both be [B, L, heads, head_dim]")
-    B, L, Hh, D = q.shape
+    Returns (q_out, k_out); with ``inplace`` the inputs are overwritten.  With
+    ``q=None`` only K is rotated (for :func:`attn_full_rope_q`) and q_out is None."""
+    if k.dim() != 4:
+        raise ValueError("k must be [B, L, heads, head_dim]")
+    B, L, Hh, D = k.shape
     Tg, Hg, Wg = grid
     if Tg * Hg * Wg != L:
         raise ValueError("grid does not match the sequence length")
     d_t, d_h, d_w = default_split(D) if split is None else split
+    qp, qop, q_out = _q_and_out(q, k, q_out, inplace)
     if inplace:
-        q_out, k_out = q, k
-    q_out = torch.empty_like(q) if q_out is None else q_out
+        k_out = k
     k_out = torch.empty_like(k) if k_out is None else k_out
     _check("vdit_rope_3d", lib().vdit_rope_3d(
-        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
-        _dev(k_out, "k_out", torch.bfloat16), B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
+        qp, _dev(k, "k", torch.bfloat16), qop, _dev(k_out, "k_out", torch.bfloat16),
+        B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
     return q_out, k_out
+
+
+def rope_3d_table(grid, head_dim: int, split=None, theta: float = 10000.0, out=None, device=None, stream=None):
+    """The 3D RoPE's (cos, sin) pairs per axis position, float32 [n, 2] on the
+    device: time [Tg][d_t/2], then height [Hg][d_h/2], then width [Wg][d_w/2]
+    (the layout ``include/vdit.h`` gives for vdit_rope_3d_table).  The input of
+    :func:`attn_full_rope_q`; it depends only on the grid, the split and theta."""
+    Tg, Hg, Wg = grid
+    d_t, d_h, d_w = default_split(head_dim) if split is None else split
+    n = lib().vdit_rope_3d_table_entries(Tg, Hg, Wg, head_dim, d_t, d_h, d_w)
+    if n < 0:
+        raise ValueError("bad grid or split")
+    if out is None:
+        out = torch.empty((max(n, 1), 2), dtype=torch.float32,
+                          device=device if device is not None else torch.device("cuda", torch.cuda.current_device()))
+    elif out.dtype != torch.float32 or out.numel() < 2 * n:
+        raise ValueError(f"out must be float32 with at least {2 * n} elements")
+    _check("vdit_rope_3d_table", lib().vdit_rope_3d_table(
+        _dev(out, "out", torch.float32), Tg, Hg, Wg, head_dim, d_t, d_h, d_w, float(theta), _stream(stream)))
+    return out[:n]
 
 
 def patch_embed_3d(latent: torch.Tensor, weight: torch.Tensor, patch=(1, 2, 2), bias=None, out=None,
@@ -210,23 +249,23 @@ def unpatchify_3d(tokens: torch.Tensor, C: int, grid, patch=(1, 2, 2), out=None,
     return out
 
 
-def qk_norm_rope_3d(q: torch.Tensor, k: torch.Tensor, grid, norm_group: int, wq=None, wk=None,
+def qk_norm_rope_3d(q: torch.Tensor | None, k: torch.Tensor, grid, norm_group: int, wq=None, wk=None,
                     eps: float = 1e-6, split=None, theta: float = 10000.0, q_out=None, k_out=None,
                     inplace: bool = False, stream=None):
     """RMSNorm of Q and K over groups of ``norm_group`` channels of each token
     (head_dim: per head; heads*head_dim: the whole token), weights ``wq``/``wk``
     (float32 [norm_group] on the device, or None for 1), then the 3D rotation of
-    :func:`rope_3d`, in one pass.  Returns (q_out, k_out)."""
-    if q.dim() != 4 or q.shape != k.shape:
-        raise ValueError("q and k must both be [B, L, heads, head_dim]")
-    B, L, Hh, D = q.shape
+    :func:`rope_3d`, in one pass.  Returns (q_out, k_out); ``q=None``: K only."""
+    if k.dim() != 4:
+        raise ValueError("k must be [B, L, heads, head_dim]")
+    B, L, Hh, D = k.shape
     Tg, Hg, Wg = grid
     if Tg * Hg * Wg != L:
         raise ValueError("grid does not match the sequence length")
     d_t, d_h, d_w = default_split(D) if split is None else split
+    qp, qop, q_out = _q_and_out(q, k, q_out, inplace)
     if inplace:
-        q_out, k_out = q, k
-    q_out = torch.empty_like(q) if q_out is None else q_out
+        k_out = k
     k_out = torch.empty_like(k) if k_out is None else k_out
     w_ptrs = []
     for w, name in ((wq, "wq"), (wk, "wk")):
@@ -237,7 +276,7 @@ def qk_norm_rope_3d(q: torch.Tensor, k: torch.Tensor, grid, norm_group: int, wq=
                 raise ValueError(f"{name} must have norm_group entries")
             w_ptrs.append(_dev(w, name, torch.float32))
     _check("vdit_qk_norm_rope_3d", lib().vdit_qk_norm_rope_3d(
-        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(q_out, "q_out", torch.bfloat16),
+        qp, _dev(k, "k", torch.bfloat16), qop,
         _dev(k_out, "k_out", torch.bfloat16), w_ptrs[0], w_ptrs[1], int(norm_group), float(eps),
         B, Tg, Hg, Wg, Hh, D, d_t, d_h, d_w, float(theta), _stream(stream)))
     return q_out, k_out
@@ -275,6 +314,32 @@ def attn_full(q, k, v, out=None, lse=None, scale: float = 0.0, stream=None):
     _check("vdit_attn_full", lib().vdit_attn_full(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, L, Hh, D,
         float(scale), _stream(stream)))
+    return out if lse_t is None else (out, lse_t)
+
+
+def attn_full_rope_q(q, k, v, grid, table, split=None, wq=None, norm_group: int = 0, eps: float = 1e-6,
+                     out=None, lse=None, scale: float = 0.0, stream=None):
+    """Full 3D self-attention with Q as projected: the kernel applies the per-head
+    RMSNorm (``norm_group`` = head_dim, weight ``wq`` float32 [head_dim] or None;
+    0: no norm) and the 3D rotation to Q in its prologue, with the pairs of
+    ``table`` (:func:`rope_3d_table` of the same grid and split).  K must already
+    be normalised and rotated (:func:`rope_3d` / :func:`qk_norm_rope_3d` with
+    ``q=None``).  ``lse=True`` also returns [B, heads, L]."""
+    out, lse_t, lse_p = _attn_io(q, k, v, out, lse)
+    B, L, Hh, D = q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != L:
+        raise ValueError("grid does not match the sequence length")
+    d_t, d_h, d_w = default_split(D) if split is None else split
+    wp = None
+    if wq is not None:
+        if tuple(wq.shape) != (D,):
+            raise ValueError("wq must have head_dim entries")
+        wp = _dev(wq, "wq", torch.float32)
+    _check("vdit_attn_full_rope_q", lib().vdit_attn_full_rope_q(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dev(out, "out", torch.bfloat16), lse_p, B, Tg, Hg, Wg, Hh, D,
+        float(scale), d_t, d_h, d_w, _dev(table, "table", torch.float32), wp, int(norm_group), float(eps),
+        _stream(stream)))
     return out if lse_t is None else (out, lse_t)
 
 

@@ -63,7 +63,7 @@ struct AttnCfg {
   static constexpr int TILE_BYTES = BM * D * 2;
   static constexpr int NK = D >= 128 ? 3 : 4;                  // K ring stages
   static constexpr int NV = D >= 128 ? 2 : (D >= 64 ? 3 : 4);  // V ring stages
-  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NQ + 1;
+  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 3 * NQ + 1;
   static constexpr int SMEM_BYTES = 1024 + (NQ + NK + NV) * TILE_BYTES + NBARS * 8 + 16;
   static constexpr int THREADS = 384;                          // three warpgroups
   static constexpr int TMA_WARP = 8, MMA_WARP = 9;
@@ -99,12 +99,21 @@ struct AttnParams {
   int n_qblocks;       // ceil(L / 256): CTAs per (sequence, head)
   int n_kv;            // ceil(Lk / 128)
   float scale_log2;    // scale * log2(e)
+  // Q normalised and rotated in the prologue (attn_fwd_tcgen05_rope_q_kernel only)
+  const float2* rope_tab;  // (cos, sin): time [Tg][pt], then height [Hg][ph], then width [Wg][pw]
+  const float* wq;         // RMSNorm weight [D], or null (weight 1)
+  int rope_hg, rope_wg;    // grid rows and columns
+  int rope_pt, rope_ph;    // pairs in the time and height segments (width: the rest)
+  int rope_off_h, rope_off_w;  // first table entry of the height and width segments
+  int rope_pw;
+  int norm;                // 1: RMSNorm over each head's D channels, then the rotation
+  float eps, inv_d;        // RMSNorm epsilon, 1/D
 };
 
 // Wait sites recorded by the watchdog.
 enum : int {
   kSiteQFull = 1, kSiteKFull, kSiteVFull, kSiteKEmpty, kSiteVEmpty, kSiteSFull, kSitePFull, kSiteODone,
-  kSiteDrain
+  kSiteDrain, kSiteQReady
 };
 
 // A wait bounded by time only (used to drain copies and MMAs before exit).
@@ -178,11 +187,109 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_
   }
 }
 
-template <int D, bool kStageO>
-__global__ void __launch_bounds__(384, 1)
-    attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                            const AttnParams p) {
+// Q/K RMSNorm and 3D RoPE of Q in the attention prologue ("How AI Generates
+// Video: Inside Sora and Wan2.1 on a Real GPU", section 5, Sub-Layer 1: Q and
+// K are RMS-normalised, then rotated by the factorised 3D RoPE of section 4,
+// then attend).  One softmax thread owns one query row of its tile: it fetches
+// the row's (cos, sin) pairs from the per-axis table while the TMA copy of Q
+// is still landing, then rewrites its row in place in the tile's swizzled
+// shared-memory copy, before the tile's first Q.K^T.  The arithmetic is that of
+// the stand-alone passes, operation for operation: the sum of squares of each
+// 8-element vector in fused multiply-adds, the vectors' sums added in the
+// butterfly order of the per-head norm pass, y = x * rsqrt(mean + eps) * w with
+// separately rounded products, the rotation with separately rounded products
+// and sums, one rounding to bf16.  So the rotated Q equals the one
+// vdit_rope_3d (or vdit_qk_norm_rope_3d with a per-head group) would have
+// written, bit for bit.  Returns false if the wait for Q ran out.
+template <int D>
+__device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* tq, uint64_t* q_full,
+                                            uint64_t* q_ready, bool active, int i, int row, int bb, int lane) {
+  using C = AttnCfg<D>;
+  constexpr int NCH = D / 8;                    // 16-byte chunks of a row
+  constexpr int CPB = C::ROWB / 16;             // chunks per staged row of one D-block
+  const bool live = active && i < p.L;          // rows past the sequence stay zero
+  float2 cs[D / 2];
+  if (live) {
+    // the row's token in its clip: full attention and space pass run over
+    // contiguous tokens, a long time pass over one site's frames
+    const long long l = p.mode == kTime ? (long long)i * p.grp + bb % p.grp : (long long)(bb % p.grp) * p.L + i;
+    const long long hw = (long long)p.rope_hg * p.rope_wg;
+    const int tt = (int)(l / hw);
+    const int rem = (int)(l - (long long)tt * hw);
+    const int hh = rem / p.rope_wg, ww = rem - hh * p.rope_wg;
+    const int bt = tt * p.rope_pt;
+    const int bh = p.rope_off_h + hh * p.rope_ph - p.rope_pt;
+    const int bw = p.rope_off_w + ww * p.rope_pw - (p.rope_pt + p.rope_ph);
+#pragma unroll
+    for (int pi = 0; pi < D / 2; ++pi) {
+      const int x = pi < p.rope_pt ? bt + pi : (pi < p.rope_pt + p.rope_ph ? bh + pi : bw + pi);
+      cs[pi] = __ldg(p.rope_tab + x);
+    }
+  }
+  bool ok = active;
+  if (ok) ok = warp_wait(q_full, 0, kSiteQFull);
+  if (ok && live) {
+    const int key = C::ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
+    auto chunk = [&](int cc) -> uint4* {
+      return reinterpret_cast<uint4*>(tq + (cc / CPB) * C::DB_BYTES + row * C::ROWB + (((cc % CPB) ^ key) << 4));
+    };
+    float nscale = 1.f;
+    if (p.norm) {
+      float a[NCH];
+#pragma unroll
+      for (int cc = 0; cc < NCH; ++cc) {
+        const uint4 x = *chunk(cc);
+        const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&u[m]);
+          const float x0 = __low2float(pr), x1 = __high2float(pr);
+          acc = fmaf(x0, x0, acc);
+          acc = fmaf(x1, x1, acc);
+        }
+        a[cc] = acc;
+      }
+#pragma unroll
+      for (int o = NCH / 2; o >= 1; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < o; ++k) a[k] = a[k] + a[k + o];
+      nscale = rsqrtf(fmaf(a[0], p.inv_d, p.eps));
+    }
+#pragma unroll
+    for (int cc = 0; cc < NCH; ++cc) {
+      uint4* dst = chunk(cc);
+      const uint4 x = *dst;
+      uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&u[m]);
+        float x0 = __low2float(pr), x1 = __high2float(pr);
+        if (p.norm) {
+          const float w0 = p.wq != nullptr ? __ldg(p.wq + cc * 8 + 2 * m) : 1.f;
+          const float w1 = p.wq != nullptr ? __ldg(p.wq + cc * 8 + 2 * m + 1) : 1.f;
+          x0 = __fmul_rn(__fmul_rn(x0, nscale), w0);
+          x1 = __fmul_rn(__fmul_rn(x1, nscale), w1);
+        }
+        const float2 c = cs[cc * 4 + m];
+        const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
+        const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
+        u[m] = pack_bf16x2(re, im);
+      }
+      *dst = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  }
+  // the rewritten rows become visible to the tensor core, then the warp reports
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (ok && lane == 0) mbar_arrive(q_ready);
+  return ok;
+}
+
+template <int D, bool kStageO, bool kRopeQ>
+__device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                              const CUtensorMap& tmV, const CUtensorMap& tmO,
+                                              const AttnParams& p) {
   using C = AttnCfg<D>;
   unsigned char* smem_raw = dyn_smem;
   const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
@@ -198,7 +305,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* s_full = v_empty + C::NV;      // [NQ]
   uint64_t* p_full = s_full + C::NQ;       // [NQ]
   uint64_t* drain = p_full + C::NQ;        // every UMMA of the CTA has finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_ready = drain + 1;           // [NQ] Q tile rotated in place (kRopeQ)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + C::NQ);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -222,6 +330,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < C::NQ; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);           // one elected lane per softmax warp
+      mbar_init(&q_ready[i], 4);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -314,11 +423,25 @@ __global__ void __launch_bounds__(384, 1)
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, kSiteQFull) && mbar_wait(&k_full[0], 0, kSiteKFull);
-      if (ok) {
-        tc_fence_after();
-        for (int i = 0; i < nq; ++i) qk(i, 0);
-        umma_commit(&k_empty[0]);
+      bool ok;
+      if constexpr (kRopeQ) {
+        // each tile's first Q.K^T waits until its softmax warps have rotated Q
+        ok = mbar_wait(&k_full[0], 0, kSiteKFull);
+        for (int i = 0; i < nq && ok; ++i) {
+          ok = mbar_wait(&q_ready[i], 0, kSiteQReady);
+          if (ok) {
+            tc_fence_after();
+            qk(i, 0);
+          }
+        }
+        if (ok) umma_commit(&k_empty[0]);
+      } else {
+        ok = mbar_wait(q_full, 0, kSiteQFull) && mbar_wait(&k_full[0], 0, kSiteKFull);
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < nq; ++i) qk(i, 0);
+          umma_commit(&k_empty[0]);
+        }
       }
       // Fixed issue order, the one the two tiles' ping-pong settles into:
       //   O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T, O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T.
@@ -365,6 +488,8 @@ __global__ void __launch_bounds__(384, 1)
     float m_use = -INFINITY;                      // max used for the exponentials (log2 units)
     float l_sum = 0.f;
     bool ok = tile < nq;
+    if constexpr (kRopeQ) ok = rope_q_rows<D>(p, sQ + tile * C::TILE_BYTES, q_full, &q_ready[tile], ok,
+                                              q0 + tile * C::BM + row, row, bb, lane);
     for (int j = 0; j < n && ok; ++j) {
       if (!warp_wait(&s_full[tile], j & 1, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
@@ -526,6 +651,26 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// Full attention, a space pass or a long time pass over Q, K and V as given.
+template <int D, bool kStageO>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_tcgen05_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                            const AttnParams p) {
+  attn_fwd_body<D, kStageO, false>(tmQ, tmK, tmV, tmO, p);
+}
+
+// The same with Q RMS-normalised (optionally) and rotated by the 3D RoPE in
+// the prologue: the caller passes Q as projected, K already normalised and
+// rotated.
+template <int D, bool kStageO>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_tcgen05_rope_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                                   const AttnParams p) {
+  attn_fwd_body<D, kStageO, true>(tmQ, tmK, tmV, tmO, p);
 }
 
 }  // namespace vdit

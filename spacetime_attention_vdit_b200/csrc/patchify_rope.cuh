@@ -200,7 +200,8 @@ __global__ void __launch_bounds__(kPatchify122Threads) patchify122_f32_kernel(co
 // 1 / theta^(2i/d) for pair i of its axis segment is built once per CTA.  Then
 // all heads of Q and K for those tokens stream through 16-byte vectors (four
 // pairs each); each pair is rotated with separately rounded float32 products
-// and sums and stored as bfloat16, round to nearest even.
+// and sums and stored as bfloat16, round to nearest even.  With one tensor
+// (K only, passed in the Q slots) the same loop covers that tensor alone.
 
 constexpr int kRopeThreads = 256;
 constexpr int kRopeTokens = 4;
@@ -213,7 +214,34 @@ struct RopeShape {
   int heads, D;       // head count, head width
   int pt_end, ph_end; // pair index where the h segment starts, and the w segment
   int d_t, d_h, d_w;
+  int ntens;          // 2: Q and K; 1: one tensor (K), passed in the Q slots
 };
+
+// Entry x of the per-axis (cos, sin) table: time [Tg][d_t/2], then height
+// [Hg][d_h/2] from off_h, then width [Wg][d_w/2] from off_w.  The angle is
+// pos * theta^(-2i/d) for pair i of a segment of width d, formed in float64;
+// cos and sin are rounded once to float32 (the snippet's complex64 cache).
+__device__ __forceinline__ float2 rope_axis_entry(int x, int off_h, int off_w, int d_t, int d_h, int d_w,
+                                                  double theta) {
+  const int pt = d_t / 2, ph = d_h / 2, pw = d_w / 2;
+  int pos, i, d;
+  if (x < off_h) { pos = x / pt; i = x - pos * pt; d = d_t; }
+  else if (x < off_w) { pos = (x - off_h) / ph; i = x - off_h - pos * ph; d = d_h; }
+  else { pos = (x - off_w) / pw; i = x - off_w - pos * pw; d = d_w; }
+  double sn, cn;
+  sincos((double)pos * (1.0 / pow(theta, (double)(2 * i) / (double)d)), &sn, &cn);
+  return make_float2((float)cn, (float)sn);
+}
+
+// The whole per-axis table in global memory, for kernels that look the pairs
+// up instead of building them (the attention kernel that rotates Q itself).
+__global__ void rope3d_table_kernel(float2* tab, int Tg, int Hg, int Wg, int d_t, int d_h, int d_w,
+                                    double theta) {
+  if (watchdog_tripped()) return;
+  const int off_h = Tg * (d_t / 2), off_w = off_h + Hg * (d_h / 2), n = off_w + Wg * (d_w / 2);
+  for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < n; x += gridDim.x * blockDim.x)
+    tab[x] = rope_axis_entry(x, off_h, off_w, d_t, d_h, d_w, theta);
+}
 
 __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat16* q_in, const __nv_bfloat16* k_in,
                                                               __nv_bfloat16* q_out, __nv_bfloat16* k_out,
@@ -253,12 +281,12 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat1
     // Each thread keeps kRopeBatch 16-byte loads in flight before rotating them.
     // Every vector is read and written by the same thread, so in-place use is safe.
     const int nvec = nt * vec_per_tok;                   // per tensor
-    for (int e0 = threadIdx.x; e0 < 2 * nvec; e0 += blockDim.x * kRopeBatch) {
+    for (int e0 = threadIdx.x; e0 < s.ntens * nvec; e0 += blockDim.x * kRopeBatch) {
       uint4 v[kRopeBatch];
 #pragma unroll
       for (int u = 0; u < kRopeBatch; ++u) {
         const int e = e0 + u * blockDim.x;
-        if (e < 2 * nvec) {
+        if (e < s.ntens * nvec) {
           const int which = e >= nvec;                   // 0: Q, 1: K
           const int ee = which ? e - nvec : e;
           const long long off = tok0 * (long long)vec_per_tok + ee;
@@ -268,7 +296,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat1
 #pragma unroll
       for (int u = 0; u < kRopeBatch; ++u) {
         const int e = e0 + u * blockDim.x;
-        if (e < 2 * nvec) {
+        if (e < s.ntens * nvec) {
           const int which = e >= nvec;
           const int ee = which ? e - nvec : e;
           const int j = ee / vec_per_tok;
@@ -312,7 +340,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat1
 // frees its stage for the copy kNormStages tokens later.  The (cos, sin) of
 // every pair at every position of its axis (Tg x d_t/2 + Hg x d_h/2 + Wg x
 // d_w/2 entries) are built once per CTA in shared memory, after the ring, so
-// that a token's rotation is a table lookup.
+// that a token's rotation is a table lookup.  With one tensor (K only) just
+// K's rows are copied and threads 0..127 only take part in the barriers.
 
 constexpr int kNormThreads = 256;
 constexpr int kNormStages = 4;
@@ -337,15 +366,8 @@ __global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
   const int pt = s.d_t / 2, ph = s.d_h / 2, pw = s.d_w / 2;
   const int Tg = (int)(s.L / ((long long)s.Hg * s.Wg));
   const int off_h = Tg * pt, off_w = off_h + s.Hg * ph, n_tab = off_w + s.Wg * pw;
-  for (int x = threadIdx.x; x < n_tab; x += blockDim.x) {
-    int pos, i, d;
-    if (x < off_h) { pos = x / pt; i = x - pos * pt; d = s.d_t; }
-    else if (x < off_w) { pos = (x - off_h) / ph; i = x - off_h - pos * ph; d = s.d_h; }
-    else { pos = (x - off_w) / pw; i = x - off_w - pos * pw; d = s.d_w; }
-    double sn, cn;
-    sincos((double)pos * (1.0 / pow(theta, (double)(2 * i) / (double)d)), &sn, &cn);
-    tab[x] = make_float2((float)cn, (float)sn);
-  }
+  for (int x = threadIdx.x; x < n_tab; x += blockDim.x)
+    tab[x] = rope_axis_entry(x, off_h, off_w, s.d_t, s.d_h, s.d_w, theta);
   if (threadIdx.x == 0) {
     for (int st = 0; st < kNormStages; ++st) mbar_init(&full[st], 1);
     fence_mbar_init();
@@ -357,8 +379,8 @@ __global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
   auto issue = [&](long long k) {                       // thread 0: token k of this CTA into its stage
     const int st = (int)(k % kNormStages);
     const long long tok = blockIdx.x + k * gridDim.x;
-    mbar_arrive_expect_tx(&full[st], 2u * row_bytes);
-    bulk_load(ring + (size_t)st * 2 * nv, q_in + tok * nv * 8, row_bytes, &full[st]);
+    mbar_arrive_expect_tx(&full[st], (uint32_t)s.ntens * row_bytes);
+    if (s.ntens == 2) bulk_load(ring + (size_t)st * 2 * nv, q_in + tok * nv * 8, row_bytes, &full[st]);
     bulk_load(ring + (size_t)st * 2 * nv + nv, k_in + tok * nv * 8, row_bytes, &full[st]);
   };
   long long issued = n_my < kNormStages ? n_my : kNormStages;
@@ -366,6 +388,7 @@ __global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
     for (long long k = 0; k < issued; ++k) issue(k);
 
   const int which = threadIdx.x >> 7;                   // 0: Q, 1: K
+  const bool active = which == 1 || s.ntens == 2;       // K only: the Q threads idle between barriers
   const int t = threadIdx.x & 127;
   const int lane = threadIdx.x & 31, wt = t >> 5;       // warp within the tensor's four
   const int gv = group / 8;                             // vectors per group
@@ -392,7 +415,7 @@ __global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
 #pragma unroll
     for (int r = 0; r < kNormVecs; ++r) {
       const int e = t + 128 * r;
-      v[r] = e < nv ? sv[e] : make_uint4(0u, 0u, 0u, 0u);
+      v[r] = (e < nv && active) ? sv[e] : make_uint4(0u, 0u, 0u, 0u);
     }
     auto vec_sq = [&](const uint4& x) -> float {
       const uint32_t u[4] = {x.x, x.y, x.z, x.w};
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(kNormThreads) qk_norm_rope3d_kernel(
         for (int o = gv >> 1; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
       }
       const int e = t + 128 * r;
-      if (e < nv) {
+      if (e < nv && active) {
         const float scale = rsqrtf(fmaf(sq, inv_group, eps));
         const int c0 = (e * 8) % group;                 // channel of the vector's first element in its group
         float wv[8];

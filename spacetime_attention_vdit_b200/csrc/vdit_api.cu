@@ -112,16 +112,21 @@ bool make_2d_map(CUtensorMap* map, const void* base, long long cols, long long r
 // Key tiles (of 128 keys) up to which the kernel stages O for TMA stores.
 constexpr int kStagedOMaxKeyTiles = 16;
 
+// `rope`: null, or the RoPE fields of AttnParams for the kernel that rotates Q
+// in its prologue.
 template <int D>
 int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq, int L,
-                   int Lk, int grp, int heads, float scale, cudaStream_t stream) {
+                   int Lk, int grp, int heads, float scale, cudaStream_t stream, const AttnParams* rope = nullptr) {
   using C = AttnCfg<D>;
   static bool smem_row[kMaxDevices] = {}, smem_staged[kMaxDevices] = {};
+  static bool smem_row_r[kMaxDevices] = {}, smem_staged_r[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!ensure_smem(attn_fwd_tcgen05_kernel<D, false>, C::SMEM_BYTES, smem_row) ||
-        !ensure_smem(attn_fwd_tcgen05_kernel<D, true>, C::SMEM_BYTES, smem_staged))
+        !ensure_smem(attn_fwd_tcgen05_kernel<D, true>, C::SMEM_BYTES, smem_staged) ||
+        !ensure_smem(attn_fwd_tcgen05_rope_q_kernel<D, false>, C::SMEM_BYTES, smem_row_r) ||
+        !ensure_smem(attn_fwd_tcgen05_rope_q_kernel<D, true>, C::SMEM_BYTES, smem_staged_r))
       return VDIT_ERR_CUDA;
   }
   // geometry of the 5-D view
@@ -153,7 +158,7 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
       !make_qkv_map(&mv, v, D, heads, sites, k_positions, batches, site_stride, pos_stride, k_batch_stride) ||
       !make_qkv_map(&mo, o, D, heads, sites, positions, batches, site_stride, pos_stride, batch_stride))
     return VDIT_ERR_CUDA;
-  AttnParams p;
+  AttnParams p = rope != nullptr ? *rope : AttnParams{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.n_seq = n_seq;
@@ -171,21 +176,43 @@ int launch_tcgen05(const void* q, const void* k, const void* v, void* o, float* 
   // give each CTA few key tiles, so its epilogue weighs: O goes out staged in
   // shared memory by TMA stores.  Long ones keep the per-row stores, whose
   // variant of the kernel runs its key-tile loop faster.
-  if (p.n_kv <= kStagedOMaxKeyTiles)
-    attn_fwd_tcgen05_kernel<D, true><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
-  else
-    attn_fwd_tcgen05_kernel<D, false><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  const bool staged = p.n_kv <= kStagedOMaxKeyTiles;
+  const unsigned g = (unsigned)grid;
+  if (rope != nullptr) {
+    if (staged)
+      attn_fwd_tcgen05_rope_q_kernel<D, true><<<g, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else
+      attn_fwd_tcgen05_rope_q_kernel<D, false><<<g, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  } else if (staged) {
+    attn_fwd_tcgen05_kernel<D, true><<<g, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  } else {
+    attn_fwd_tcgen05_kernel<D, false><<<g, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  }
   return last_launch_status();
 }
 
 int dispatch_tcgen05(int D, const void* q, const void* k, const void* v, void* o, float* lse, int mode, int n_seq,
-                     int L, int Lk, int grp, int heads, float scale, cudaStream_t stream) {
+                     int L, int Lk, int grp, int heads, float scale, cudaStream_t stream,
+                     const AttnParams* rope = nullptr) {
   switch (D) {
-    case 32: return launch_tcgen05<32>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
-    case 64: return launch_tcgen05<64>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
-    case 128: return launch_tcgen05<128>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream);
+    case 32: return launch_tcgen05<32>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream, rope);
+    case 64: return launch_tcgen05<64>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream, rope);
+    case 128: return launch_tcgen05<128>(q, k, v, o, lse, mode, n_seq, L, Lk, grp, heads, scale, stream, rope);
     default: return VDIT_ERR_UNSUPPORTED;
   }
+}
+
+// Checks shared by the RoPE calls: grid, split and theta.
+int check_rope_shape(int Tg, int Hg, int Wg, int head_dim, int d_t, int d_h, int d_w, float theta) {
+  if (Tg <= 0 || Hg <= 0 || Wg <= 0 || head_dim <= 0) return VDIT_ERR_SHAPE;
+  if (d_t < 0 || d_h < 0 || d_w < 0 || (d_t | d_h | d_w) & 1 || d_t + d_h + d_w != head_dim) return VDIT_ERR_SHAPE;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return VDIT_ERR_SHAPE;
+  if ((long long)Tg * Hg * Wg > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  return VDIT_OK;
+}
+
+long long rope_table_entries(int Tg, int Hg, int Wg, int d_t, int d_h, int d_w) {
+  return (long long)Tg * (d_t / 2) + (long long)Hg * (d_h / 2) + (long long)Wg * (d_w / 2);
 }
 
 template <int D, int TB>
@@ -255,7 +282,7 @@ int check_attn_args(const void* q, const void* k, const void* v, const void* o, 
 
 extern "C" {
 
-int vdit_version(void) { return 10000; }
+int vdit_version(void) { return 10100; }
 
 const char* vdit_status_string(int status) {
   switch (status) {
@@ -427,6 +454,8 @@ int vdit_patch_embed_3d(const float* latent, const void* weight, const float* bi
 
 int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, int B, int Tg, int Hg, int Wg,
                  int heads, int head_dim, int d_t, int d_h, int d_w, float theta, vdit_stream_t stream) {
+  const bool k_only = q_in == nullptr && q_out == nullptr;
+  if (k_only) { q_in = k_in; q_out = k_out; }
   if (!q_in || !k_in || !q_out || !k_out) return VDIT_ERR_NULL;
   if (B <= 0 || Tg <= 0 || Hg <= 0 || Wg <= 0 || heads <= 0 || head_dim <= 0) return VDIT_ERR_SHAPE;
   if (d_t < 0 || d_h < 0 || d_w < 0 || (d_t | d_h | d_w) & 1 || d_t + d_h + d_w != head_dim) return VDIT_ERR_SHAPE;
@@ -441,6 +470,7 @@ int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, i
   s.heads = heads; s.D = head_dim;
   s.pt_end = d_t / 2; s.ph_end = (d_t + d_h) / 2;
   s.d_t = d_t; s.d_h = d_h; s.d_w = d_w;
+  s.ntens = k_only ? 1 : 2;
   const long long want = (s.ntok + kRopeTokens - 1) / kRopeTokens;
   const long long cap = (long long)sm_count() * 8;
   const unsigned grid = (unsigned)(want < cap ? want : cap);
@@ -453,6 +483,8 @@ int vdit_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, i
 int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* wq,
                          const float* wk, int norm_group, float eps, int B, int Tg, int Hg, int Wg, int heads,
                          int head_dim, int d_t, int d_h, int d_w, float theta, vdit_stream_t stream) {
+  const bool k_only = q_in == nullptr && q_out == nullptr;
+  if (k_only) { q_in = k_in; q_out = k_out; }
   if (!q_in || !k_in || !q_out || !k_out) return VDIT_ERR_NULL;
   if (B <= 0 || Tg <= 0 || Hg <= 0 || Wg <= 0 || heads <= 0 || head_dim <= 0) return VDIT_ERR_SHAPE;
   if (d_t < 0 || d_h < 0 || d_w < 0 || (d_t | d_h | d_w) & 1 || d_t + d_h + d_w != head_dim) return VDIT_ERR_SHAPE;
@@ -475,6 +507,7 @@ int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* 
   s.heads = heads; s.D = head_dim;
   s.pt_end = d_t / 2; s.ph_end = (d_t + d_h) / 2;
   s.d_t = d_t; s.d_h = d_h; s.d_w = d_w;
+  s.ntens = k_only ? 1 : 2;
   const long long cap = (long long)sm_count() * 2;
   const unsigned grid = (unsigned)(s.ntok < cap ? s.ntok : cap);
   // the ring (Q and K rows of kNormStages tokens) and the per-axis (cos, sin) tables
@@ -509,6 +542,56 @@ int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* 
   if (rc != VDIT_OK) return rc;
   return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, L, L, 1, heads, resolve_scale(scale, head_dim),
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+long long vdit_rope_3d_table_entries(int Tg, int Hg, int Wg, int head_dim, int d_t, int d_h, int d_w) {
+  if (check_rope_shape(Tg, Hg, Wg, head_dim, d_t, d_h, d_w, 1.f) != VDIT_OK) return -1;
+  return rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w);
+}
+
+int vdit_rope_3d_table(float* table, int Tg, int Hg, int Wg, int head_dim, int d_t, int d_h, int d_w, float theta,
+                       vdit_stream_t stream) {
+  if (!table) return VDIT_ERR_NULL;
+  const int rc = check_rope_shape(Tg, Hg, Wg, head_dim, d_t, d_h, d_w, theta);
+  if (rc != VDIT_OK) return rc;
+  if (!aligned16(table)) return VDIT_ERR_ALIGN;
+  const long long n = rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w);
+  if (n > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  if (n == 0) return VDIT_OK;
+  const long long blocks = (n + 255) / 256;
+  const long long cap = (long long)sm_count() * 4;
+  rope3d_table_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<float2*>(table), Tg, Hg, Wg, d_t, d_h, d_w, (double)theta);
+  return last_launch_status();
+}
+
+int vdit_attn_full_rope_q(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Tg, int Hg,
+                          int Wg, int heads, int head_dim, float scale, int d_t, int d_h, int d_w,
+                          const float* rope_table, const float* wq, int norm_group, float eps,
+                          vdit_stream_t stream) {
+  if (!rope_table) return VDIT_ERR_NULL;
+  if (Tg <= 0 || Hg <= 0 || Wg <= 0) return (!q || !k || !v || !o) ? VDIT_ERR_NULL : VDIT_ERR_SHAPE;
+  const long long L = (long long)Tg * Hg * Wg;
+  int rc = check_attn_args(q, k, v, o, lse, B, L, heads, head_dim);
+  if (rc != VDIT_OK) return rc;
+  rc = check_rope_shape(Tg, Hg, Wg, head_dim, d_t, d_h, d_w, 1.f);
+  if (rc != VDIT_OK) return rc;
+  if (norm_group != 0 && norm_group != head_dim) return VDIT_ERR_UNSUPPORTED;
+  if (norm_group != 0 && (!(eps >= 0.f) || !std::isfinite(eps))) return VDIT_ERR_SHAPE;
+  if (!aligned16(rope_table) || (wq && !aligned16(wq))) return VDIT_ERR_ALIGN;
+  if (rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w) > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  AttnParams r{};
+  r.rope_tab = reinterpret_cast<const float2*>(rope_table);
+  r.wq = wq;
+  r.rope_hg = Hg; r.rope_wg = Wg;
+  r.rope_pt = d_t / 2; r.rope_ph = d_h / 2; r.rope_pw = d_w / 2;
+  r.rope_off_h = Tg * (d_t / 2);
+  r.rope_off_w = r.rope_off_h + Hg * (d_h / 2);
+  r.norm = norm_group != 0;
+  r.eps = eps;
+  r.inv_d = 1.f / (float)head_dim;
+  return dispatch_tcgen05(head_dim, q, k, v, o, lse, kSeq, B, (int)L, (int)L, 1, heads,
+                          resolve_scale(scale, head_dim), reinterpret_cast<cudaStream_t>(stream), &r);
 }
 
 int vdit_attn_cross(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq, int Lk,

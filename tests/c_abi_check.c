@@ -24,7 +24,7 @@ int main(void) {
   void* const fake = (void*)(uintptr_t)0x7f0000000000ull;
   void* const mis = (void*)(uintptr_t)(0x7f0000000000ull + 8);
 
-  if (vdit_version() != 10000) { printf("FAIL version %d\n", vdit_version()); ++fails; }
+  if (vdit_version() != 10100) { printf("FAIL version %d\n", vdit_version()); ++fails; }
   for (int s = 0; s <= VDIT_ERR_TIMEOUT; ++s)
     if (vdit_status_string(s) == NULL || strlen(vdit_status_string(s)) == 0) {
       printf("FAIL status string %d\n", s);
@@ -61,5 +61,23 @@ int main(void) {
          vdit_attn_cross(fake, fake, fake, fake, (float*)((char*)fake + 2), 1, 256, 77, 2, 128, 0.f, NULL),
          VDIT_ERR_ALIGN);
   expect("watchdog self-test site", vdit_watchdog_selftest(0, NULL), VDIT_ERR_SHAPE);
+  expect("rope K only", vdit_rope_3d(NULL, fake, NULL, mis, 1, 5, 30, 52, 40, 128, 44, 42, 42, 10000.f, NULL),
+         VDIT_ERR_ALIGN);
+  expect("rope half Q", vdit_rope_3d(NULL, fake, fake, fake, 1, 5, 30, 52, 40, 128, 44, 42, 42, 10000.f, NULL),
+         VDIT_ERR_NULL);
+  if (vdit_rope_3d_table_entries(21, 30, 52, 128, 44, 42, 42) != 2184) {
+    printf("FAIL table entries\n");
+    ++fails;
+  }
+  expect("table split", vdit_rope_3d_table((float*)fake, 21, 30, 52, 128, 44, 42, 40, 10000.f, NULL),
+         VDIT_ERR_SHAPE);
+  expect("rope-q table null",
+         vdit_attn_full_rope_q(fake, fake, fake, fake, NULL, 1, 5, 30, 52, 40, 128, 0.f, 44, 42, 42, NULL, NULL, 0,
+                               1e-6f, NULL),
+         VDIT_ERR_NULL);
+  expect("rope-q token group",
+         vdit_attn_full_rope_q(fake, fake, fake, fake, NULL, 1, 5, 30, 52, 40, 128, 0.f, 44, 42, 42, (float*)fake,
+                               NULL, 5120, 1e-6f, NULL),
+         VDIT_ERR_UNSUPPORTED);
   return fails;
 }

@@ -27,19 +27,20 @@ def L():
 def declared_functions():
     with open(os.path.join(ROOT, "include", "vdit.h")) as fh:
         text = fh.read()
-    return sorted(set(re.findall(r"^(?:int|const char\*)\s+(vdit_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^(?:int|long long|const char\*)\s+(vdit_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_exports_every_declared_symbol(L):
     names = declared_functions()
     assert {"vdit_patchify_3d", "vdit_rope_3d", "vdit_attn_full", "vdit_attn_divided_time",
-            "vdit_attn_divided_space", "vdit_status_string", "vdit_device_status", "vdit_version"} <= set(names)
+            "vdit_attn_divided_space", "vdit_status_string", "vdit_device_status", "vdit_version",
+            "vdit_rope_3d_table", "vdit_rope_3d_table_entries", "vdit_attn_full_rope_q"} <= set(names)
     for n in names:
         assert hasattr(L, n), n
 
 
 def test_version_and_strings(L):
-    assert L.vdit_version() == 10000
+    assert L.vdit_version() == 10100
     for s in range(7):
         assert len(L.vdit_status_string(s)) > 0
     assert L.vdit_status_string(99) == b"unknown status"
@@ -76,6 +77,55 @@ def test_rope_validation(L):
     assert rope(L, D=36, split=(12, 12, 12)) == UNSUP  # not a multiple of 8
     assert rope(L, q=MIS) == ALIGN
     assert rope(L, ko=MIS) == ALIGN
+
+
+def test_rope_k_only_form(L):
+    """Q's pointers both NULL rotate K alone; only one of them NULL is an error."""
+    assert rope(L, q=None, qo=None, k=None) == NULL
+    assert rope(L, qo=None) == NULL
+    assert rope(L, q=None, qo=None, split=(44, 42, 40)) == SHAPE
+    assert rope(L, q=None, qo=None, ko=MIS) == ALIGN
+    assert norm_rope(L, q=None, qo=None, k=None) == NULL
+    assert norm_rope(L, q=None) == NULL
+    assert norm_rope(L, q=None, qo=None, group=96) == SHAPE
+    assert norm_rope(L, q=None, qo=None, ko=MIS) == ALIGN
+
+
+def table(L, t=FAKE, Tg=21, Hg=30, Wg=52, D=128, split=(44, 42, 42), theta=10000.0):
+    return L.vdit_rope_3d_table(t, Tg, Hg, Wg, D, *split, ctypes.c_float(theta), None)
+
+
+def test_rope_table_validation(L):
+    assert L.vdit_rope_3d_table_entries(21, 30, 52, 128, 44, 42, 42) == 21 * 22 + 30 * 21 + 52 * 21
+    assert L.vdit_rope_3d_table_entries(21, 30, 52, 128, 0, 64, 64) == 30 * 32 + 52 * 32
+    assert L.vdit_rope_3d_table_entries(21, 30, 52, 128, 44, 42, 40) == -1
+    assert L.vdit_rope_3d_table_entries(0, 30, 52, 128, 44, 42, 42) == -1
+    assert table(L, t=None) == NULL
+    assert table(L, split=(43, 43, 42)) == SHAPE
+    assert table(L, Wg=0) == SHAPE
+    assert table(L, theta=-1.0) == SHAPE
+    assert table(L, t=MIS) == ALIGN
+
+
+def attn_rope(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, grid=(3, 8, 12), heads=2, D=128,
+              split=(44, 42, 42), tab=FAKE, wq=None, group=0, eps=1e-6):
+    return L.vdit_attn_full_rope_q(q, k, v, o, lse, B, *grid, heads, D, ctypes.c_float(0.0), *split, tab, wq,
+                                   group, ctypes.c_float(eps), None)
+
+
+def test_attn_full_rope_q_validation(L):
+    assert attn_rope(L, tab=None) == NULL
+    assert attn_rope(L, q=None) == NULL
+    assert attn_rope(L, grid=(3, 0, 12)) == SHAPE
+    assert attn_rope(L, B=0) == SHAPE
+    assert attn_rope(L, split=(44, 42, 40)) == SHAPE
+    assert attn_rope(L, D=48, split=(16, 16, 16)) == UNSUP
+    assert attn_rope(L, group=256) == UNSUP           # a token-wide group needs every head
+    assert attn_rope(L, group=64) == UNSUP
+    assert attn_rope(L, group=128, eps=-1.0) == SHAPE
+    assert attn_rope(L, tab=MIS) == ALIGN
+    assert attn_rope(L, group=128, wq=MIS) == ALIGN
+    assert attn_rope(L, k=MIS) == ALIGN
 
 
 def norm_rope(L, q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, wq=None, wk=None, group=128, eps=1e-6, B=1, Tg=2, Hg=3,
@@ -194,7 +244,7 @@ def test_register_budget_fits_each_sm_subpartition(tmp_path):
         m = re.search(r"Used (\d+) registers", line)
         if m and name:
             regs[name] = int(m.group(1))
-    threads = {"attn_fwd_tcgen05_kernel": 384, "rope3d_kernel": 256, "patchify3d_kernel": 256,
+    threads = {"attn_fwd_tcgen05": 384, "rope3d_table_kernel": 256, "rope3d_kernel": 256, "patchify3d_kernel": 256,
                "patchify122_f32_kernel": 128, "qk_norm_rope3d_kernel": 256, "patch_embed_kernel": 320,
                "unpatchify3d_kernel": 256, "watchdog_selftest_kernel": 32}
 
@@ -220,7 +270,7 @@ def test_register_budget_fits_each_sm_subpartition(tmp_path):
     assert 2 * 128 * soft + 128 * ctrl <= 384 * launch
     assert 32 * (2 * soft + ctrl) <= 16384              # one warp of each warpgroup per sub-partition
     for kname, r in regs.items():
-        if "attn_fwd_tcgen05_kernel" in kname:
+        if "attn_fwd_tcgen05" in kname:
             assert r == launch, (kname, r)
         warps = block_of(kname) // 32
         per_sub = -(-warps // 4)                  # warps on the fullest sub-partition
