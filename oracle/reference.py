@@ -149,13 +149,14 @@ def rope_tables(grid, split, theta: float = 10000.0, tokens=None):
 
 def rope_axis_phasors(grid, split, theta: float = 10000.0) -> np.ndarray:
     """The RoPE's unit phasors per axis position, float64 [n, 2] of (cos, sin):
-    the Tg*d_t/2 time entries (frame-major, then pair), then Hg*d_h/2 height
-    entries, then Wg*d_w/2 width entries.  The towardsai snippet builds one
-    frequency table per axis and looks each token's angles up by its t, h and w
-    (section 4); this is that per-axis cache, before the lookup."""
+    the d_t/2 x Tg time entries (pair-major: entry i*Tg + t'), then d_h/2 x Hg
+    height entries, then d_w/2 x Wg width entries.  The towardsai snippet builds
+    one frequency table per axis and looks each token's angles up by its t, h
+    and w (section 4); this is that per-axis cache, before the lookup.  The
+    order of entries is the library's layout, which the pages do not fix."""
     parts = []
     for n, d in zip(grid, split):
-        ang = np.outer(np.arange(n, dtype=np.float64), rope_inv_freq(d, theta))   # [n, d/2]
+        ang = np.outer(rope_inv_freq(d, theta), np.arange(n, dtype=np.float64))   # [d/2, n]
         parts.append(np.stack([np.cos(ang), np.sin(ang)], axis=-1).reshape(-1, 2))
     return np.concatenate(parts, axis=0)
 

@@ -180,9 +180,10 @@ ROPE_PINS = [pin_rope_onehot, pin_rope_complex, pin_rope_relative, pin_rope_norm
 # each token's angles looked up by its t, h and w).
 
 def _phasor_index(grid, split, axis, pos, i):
-    """Row of the per-axis table: time block, then height, then width."""
+    """Row of the per-axis table: time block, then height, then width; within a
+    block pair-major (entry i * extent + pos)."""
     start = sum(grid[a] * (split[a] // 2) for a in range(axis))
-    return start + pos * (split[axis] // 2) + i
+    return start + i * grid[axis] + pos
 
 
 def pin_phasors_brute(phasors):

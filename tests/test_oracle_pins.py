@@ -241,13 +241,16 @@ def test_unpatchify_mistake_caught():
     assert _fails(pins.UNPATCHIFY_PINS, unpatchify_spatial_swapped) == 1
 
 
-def _phasor_variant(grid, split, theta=10000.0, axis_order=(0, 1, 2), swap=False, head_width=None, start=0):
+def _phasor_variant(grid, split, theta=10000.0, axis_order=(0, 1, 2), swap=False, head_width=None, start=0,
+                    pos_major=False):
     parts = []
     for a in axis_order:
         n, d = grid[a], split[a]
         j = np.arange(0, d, 2, dtype=np.float64)
         f = 1.0 / (theta ** (j / (head_width or d)))
-        ang = np.outer(np.arange(start, start + n, dtype=np.float64), f)
+        ang = np.outer(f, np.arange(start, start + n, dtype=np.float64))
+        if pos_major:
+            ang = ang.T
         c, s_ = np.cos(ang), np.sin(ang)
         parts.append(np.stack([s_, c] if swap else [c, s_], axis=-1).reshape(-1, 2))
     return np.concatenate(parts, axis=0)
@@ -258,7 +261,8 @@ def _phasor_variant(grid, split, theta=10000.0, axis_order=(0, 1, 2), swap=False
     dict(swap=True),                 # (sin, cos) instead of (cos, sin)
     dict(head_width=128),            # frequencies from the head width
     dict(start=1),                   # positions counted from 1
-], ids=["axis-order", "sin-cos", "head-width-freq", "one-based"])
+    dict(pos_major=True),            # position-major within an axis
+], ids=["axis-order", "sin-cos", "head-width-freq", "one-based", "pos-major"])
 def test_phasor_mistakes_caught(kw):
     for pin in pins.PHASOR_PINS:
         pin(_phasor_variant)
