@@ -215,10 +215,11 @@ int vdit_qk_norm_rope_3d(const void* q_in, const void* k_in, void* q_out, void* 
  * them as a cache].
  *
  * table: device float32 [n][2], n = Tg*(d_t/2) + Hg*(d_h/2) + Wg*(d_w/2)
- * (vdit_rope_3d_table_entries), 16-byte aligned, written by the call:
- *   entry t'*(d_t/2) + i                          time pair i at frame t'
- *   entry Tg*(d_t/2) + h'*(d_h/2) + i             height pair i at row h'
- *   entry Tg*(d_t/2) + Hg*(d_h/2) + w'*(d_w/2) + i  width pair i at column w'
+ * (vdit_rope_3d_table_entries), 16-byte aligned, written by the call, pair-major
+ * within each axis (neighbouring positions of one pair are neighbouring entries):
+ *   entry i*Tg + t'                               time pair i at frame t'
+ *   entry Tg*(d_t/2) + i*Hg + h'                  height pair i at row h'
+ *   entry Tg*(d_t/2) + Hg*(d_h/2) + i*Wg + w'     width pair i at column w'
  * each holding (cos a, sin a) of a = pos * theta^(-2i/d) for its segment width
  * d, formed in float64 and rounded once to float32: the values vdit_rope_3d
  * rotates with.  The table depends only on the grid, the split and theta; it

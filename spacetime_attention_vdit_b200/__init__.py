@@ -184,8 +184,9 @@ def rope_3d(q: torch.Tensor | None, k: torch.Tensor, grid, split=None, theta: fl
 
 def rope_3d_table(grid, head_dim: int, split=None, theta: float = 10000.0, out=None, device=None, stream=None):
     """The 3D RoPE's (cos, sin) pairs per axis position, float32 [n, 2] on the
-    device: time [Tg][d_t/2], then height [Hg][d_h/2], then width [Wg][d_w/2]
-    (the layout ``include/vdit.h`` gives for vdit_rope_3d_table).  The input of
+    device, pair-major within each axis: time [d_t/2][Tg], then height
+    [d_h/2][Hg], then width [d_w/2][Wg] (the layout ``include/vdit.h`` gives for
+    vdit_rope_3d_table).  The input of
     :func:`attn_full_rope_q`; it depends only on the grid, the split and theta."""
     Tg, Hg, Wg = grid
     d_t, d_h, d_w = default_split(head_dim) if split is None else split

@@ -100,12 +100,12 @@ struct AttnParams {
   int n_kv;            // ceil(Lk / 128)
   float scale_log2;    // scale * log2(e)
   // Q normalised and rotated in the prologue (attn_fwd_tcgen05_rope_q_kernel only)
-  const float2* rope_tab;  // (cos, sin): time [Tg][pt], then height [Hg][ph], then width [Wg][pw]
+  const float2* rope_tab;  // (cos, sin), pair-major: time [pt][Tg], height [ph][Hg], width [pw][Wg]
   const float* wq;         // RMSNorm weight [D], or null (weight 1)
-  int rope_hg, rope_wg;    // grid rows and columns
+  int rope_tg, rope_hg, rope_wg;  // grid frames, rows and columns
   int rope_pt, rope_ph;    // pairs in the time and height segments (width: the rest)
   int rope_off_h, rope_off_w;  // first table entry of the height and width segments
-  int rope_pw;
+  int rope_n;              // table entries (at most TILE_BYTES / 8: it is staged in V's second stage)
   int norm;                // 1: RMSNorm over each head's D channels, then the rotation
   float eps, inv_d;        // RMSNorm epsilon, 1/D
 };
@@ -190,10 +190,15 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_
 // Q/K RMSNorm and 3D RoPE of Q in the attention prologue ("How AI Generates
 // Video: Inside Sora and Wan2.1 on a Real GPU", section 5, Sub-Layer 1: Q and
 // K are RMS-normalised, then rotated by the factorised 3D RoPE of section 4,
-// then attend).  One softmax thread owns one query row of its tile: it fetches
-// the row's (cos, sin) pairs from the per-axis table while the TMA copy of Q
-// is still landing, then rewrites its row in place in the tile's swizzled
-// shared-memory copy, before the tile's first Q.K^T.  The arithmetic is that of
+// then attend).  While the TMA copy of Q is still landing, the 256 softmax
+// threads copy the per-axis (cos, sin) table into V's second ring stage (free
+// until the producer's second V load, which waits for both tiles' Q) with
+// coalesced loads and meet at a named barrier; fetching each row's 64 pairs
+// from global memory instead took several thousand cycles per CTA.  Then one
+// softmax thread owns one query row of its tile and rewrites it in place in
+// the tile's swizzled shared-memory copy, before the tile's first Q.K^T.  The
+// table is pair-major, so the 32 rows of a warp, consecutive tokens, read
+// neighbouring entries for each pair (no bank conflicts).  The arithmetic is that of
 // the stand-alone passes, operation for operation: the sum of squares of each
 // 8-element vector in fused multiply-adds, the vectors' sums added in the
 // butterfly order of the per-head norm pass, y = x * rsqrt(mean + eps) * w with
@@ -202,29 +207,29 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&s)[4][32], uint32_t t_
 // vdit_rope_3d (or vdit_qk_norm_rope_3d with a per-head group) would have
 // written, bit for bit.  Returns false if the wait for Q ran out.
 template <int D>
-__device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* tq, uint64_t* q_full,
+__device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* tq, float2* tabs, uint64_t* q_full,
                                             uint64_t* q_ready, bool active, int i, int row, int bb, int lane) {
   using C = AttnCfg<D>;
   constexpr int NCH = D / 8;                    // 16-byte chunks of a row
   constexpr int CPB = C::ROWB / 16;             // chunks per staged row of one D-block
   const bool live = active && i < p.L;          // rows past the sequence stay zero
-  float2 cs[D / 2];
+  // every softmax thread takes part, whatever its tile: the barrier counts 256
+  for (int x = (int)threadIdx.x; x < p.rope_n; x += 256) tabs[x] = __ldg(p.rope_tab + x);
+  named_bar_sync(3, 256);
+  int bt = 0, bh = 0, bw = 0;
   if (live) {
-    // the row's token in its clip: full attention and space pass run over
-    // contiguous tokens, a long time pass over one site's frames
-    const long long l = p.mode == kTime ? (long long)i * p.grp + bb % p.grp : (long long)(bb % p.grp) * p.L + i;
-    const long long hw = (long long)p.rope_hg * p.rope_wg;
-    const int tt = (int)(l / hw);
-    const int rem = (int)(l - (long long)tt * hw);
-    const int hh = rem / p.rope_wg, ww = rem - hh * p.rope_wg;
-    const int bt = tt * p.rope_pt;
-    const int bh = p.rope_off_h + hh * p.rope_ph - p.rope_pt;
-    const int bw = p.rope_off_w + ww * p.rope_pw - (p.rope_pt + p.rope_ph);
-#pragma unroll
-    for (int pi = 0; pi < D / 2; ++pi) {
-      const int x = pi < p.rope_pt ? bt + pi : (pi < p.rope_pt + p.rope_ph ? bh + pi : bw + pi);
-      cs[pi] = __ldg(p.rope_tab + x);
-    }
+    // the row's token in its clip (full attention and space pass: contiguous
+    // tokens; a long time pass: one site's frames); below 2^31 by the host's
+    // size checks
+    const uint32_t l = p.mode == kTime ? (uint32_t)i * (uint32_t)p.grp + (uint32_t)(bb % p.grp)
+                                       : (uint32_t)(bb % p.grp) * (uint32_t)p.L + (uint32_t)i;
+    const uint32_t hw = (uint32_t)p.rope_hg * (uint32_t)p.rope_wg;
+    const uint32_t tt = l / hw, rem = l - tt * hw;
+    const uint32_t hh = rem / (uint32_t)p.rope_wg, ww = rem - hh * (uint32_t)p.rope_wg;
+    // entry of pair pi: base + pi * (its axis's extent)
+    bt = (int)tt;
+    bh = p.rope_off_h + (int)hh - p.rope_pt * p.rope_hg;
+    bw = p.rope_off_w + (int)ww - (p.rope_pt + p.rope_ph) * p.rope_wg;
   }
   bool ok = active;
   if (ok) ok = warp_wait(q_full, 0, kSiteQFull);
@@ -271,7 +276,9 @@ __device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* 
           x0 = __fmul_rn(__fmul_rn(x0, nscale), w0);
           x1 = __fmul_rn(__fmul_rn(x1, nscale), w1);
         }
-        const float2 c = cs[cc * 4 + m];
+        const int pi = cc * 4 + m;
+        const float2 c = tabs[pi < p.rope_pt ? bt + pi * p.rope_tg
+                                             : (pi < p.rope_pt + p.rope_ph ? bh + pi * p.rope_hg : bw + pi * p.rope_wg)];
         const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
         const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
         u[m] = pack_bf16x2(re, im);
@@ -279,10 +286,14 @@ __device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* 
       *dst = make_uint4(u[0], u[1], u[2], u[3]);
     }
   }
-  // the rewritten rows become visible to the tensor core, then the warp reports
+  // the rewritten rows, and this thread's share of the table copy, are ordered
+  // before the tensor core's reads and the TMA's next writes there; then the
+  // warp reports (a warp of a tile past the sequence too, since the producer
+  // waits for all eight before it overwrites the table; not a warp whose wait
+  // for Q ran out, so that nothing reads a Q that may not have landed)
   fence_proxy_async_smem();
   __syncwarp();
-  if (ok && lane == 0) mbar_arrive(q_ready);
+  if ((ok || !active) && lane == 0) mbar_arrive(q_ready);
   return ok;
 }
 
@@ -291,9 +302,7 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
                                               const CUtensorMap& tmV, const CUtensorMap& tmO,
                                               const AttnParams& p) {
   using C = AttnCfg<D>;
-  unsigned char* smem_raw = dyn_smem;
-  const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
-  unsigned char* sQ = reinterpret_cast<unsigned char*>(base);      // NQ tiles
+  unsigned char* sQ = smem_base_1024();                            // NQ tiles
   unsigned char* sK = sQ + C::NQ * C::TILE_BYTES;                  // NK tiles
   unsigned char* sV = sK + C::NK * C::TILE_BYTES;                  // NV tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + C::NV * C::TILE_BYTES);
@@ -387,6 +396,12 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
       bool ok = load_k(0);
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n) ok = load_k(j + 1);
+        if constexpr (kRopeQ) {
+          // V's second stage holds the RoPE table until all eight softmax warps
+          // are done with it
+          if (j == 1)
+            for (int i = 0; i < C::NQ && ok; ++i) ok = mbar_wait(&q_ready[i], 0, kSiteQReady);
+        }
         if (ok) ok = load_v(j);
       }
       // No copy may still be landing in shared memory when the CTA exits.
@@ -425,16 +440,16 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
       };
       bool ok;
       if constexpr (kRopeQ) {
-        // each tile's first Q.K^T waits until its softmax warps have rotated Q
+        // the first Q.K^T products wait until the softmax warps have rotated
+        // Q; both tiles' are then issued back to back, as when Q lands, which
+        // starts the two tiles' ping-pong at the offset the loop runs fastest at
         ok = mbar_wait(&k_full[0], 0, kSiteKFull);
-        for (int i = 0; i < nq && ok; ++i) {
-          ok = mbar_wait(&q_ready[i], 0, kSiteQReady);
-          if (ok) {
-            tc_fence_after();
-            qk(i, 0);
-          }
+        for (int i = 0; i < nq && ok; ++i) ok = mbar_wait(&q_ready[i], 0, kSiteQReady);
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < nq; ++i) qk(i, 0);
+          umma_commit(&k_empty[0]);
         }
-        if (ok) umma_commit(&k_empty[0]);
       } else {
         ok = mbar_wait(q_full, 0, kSiteQFull) && mbar_wait(&k_full[0], 0, kSiteKFull);
         if (ok) {
@@ -488,8 +503,9 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
     float m_use = -INFINITY;                      // max used for the exponentials (log2 units)
     float l_sum = 0.f;
     bool ok = tile < nq;
-    if constexpr (kRopeQ) ok = rope_q_rows<D>(p, sQ + tile * C::TILE_BYTES, q_full, &q_ready[tile], ok,
-                                              q0 + tile * C::BM + row, row, bb, lane);
+    if constexpr (kRopeQ)
+      ok = rope_q_rows<D>(p, sQ + tile * C::TILE_BYTES, reinterpret_cast<float2*>(sV + C::TILE_BYTES), q_full,
+                          &q_ready[tile], ok, q0 + tile * C::BM + row, row, bb, lane);
     for (int j = 0; j < n && ok; ++j) {
       if (!warp_wait(&s_full[tile], j & 1, kSiteSFull)) { ok = false; break; }
       tc_fence_after();

@@ -98,8 +98,7 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
                            const __grid_constant__ CUtensorMap tmV, const TimeParams p) {
   using C = TimeCfg<D, TB>;
   constexpr int TP = C::TP;
-  const uintptr_t base = (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023);
-  unsigned char* stages = reinterpret_cast<unsigned char*>(base);
+  unsigned char* stages = smem_base_1024();
   uint64_t* full = reinterpret_cast<uint64_t*>(stages + C::NSTAGE * C::STAGE_BYTES);
   uint64_t* empty = full + C::NSTAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,15 +125,18 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       int issued = 0;
+      // (head, site, batch) of problem u = ((b * HW + s) * heads + h): divided
+      // out once, then stepped, so the issue loop carries no division
+      int h = (int)(u_begin % p.heads), s, b;
+      {
+        const long long bs = u_begin / p.heads;
+        s = (int)(bs % p.HW);
+        b = (int)(bs / p.HW);
+      }
       for (int k = 0; k < n_local; ++k) {
         const int st = (k % C::NP) * 2 + ((k / C::NP) & 1);
         const int use = k / (2 * C::NP);                    // earlier fills of this stage
         if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, 20)) break;
-        const long long u = u_begin + k;
-        const int h = (int)(u % p.heads);
-        const long long bs = u / p.heads;
-        const int s = (int)(bs % p.HW);
-        const int b = (int)(bs / p.HW);
         unsigned char* sb = stages + st * C::STAGE_BYTES;
         mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
 #pragma unroll
@@ -144,6 +146,10 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
           tma_load_5d(sb + 2 * C::TENSOR_BYTES + db * C::REGION, &tmV, &full[st], db * C::DBLK, h, s, 0, b);
         }
         issued = k + 1;
+        if (++h == p.heads) {
+          h = 0;
+          if (++s == p.HW) { s = 0; ++b; }
+        }
       }
       // drain: the last fill of every stage has landed before the CTA exits
       for (int k = issued - 2 * C::NP < 0 ? 0 : issued - 2 * C::NP; k < issued; ++k) {
@@ -164,6 +170,13 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
   const int g8 = lane >> 2;                  // fragment row within an 8-row group
   const int q2 = (lane & 3) * 2;             // fragment column pair
   int j = 0;                                 // this group's problem count
+  // (head, site, batch) of this group's first problem, then stepped by NP
+  int h = (int)((u_begin + cg) % p.heads), s, b;
+  {
+    const long long bs = (u_begin + cg) / p.heads;
+    s = (int)(bs % p.HW);
+    b = (int)(bs / p.HW);
+  }
   for (int k = cg; k < n_local; k += C::NP, ++j) {
     const int st = cg * 2 + (j & 1);
     // every lane of the warp leaves together: the loop body is full of
@@ -171,11 +184,6 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
     if (!warp_wait(&full[st], (j >> 1) & 1, 22)) break;
     unsigned char* sb = stages + st * C::STAGE_BYTES;
     const uint32_t aQ = smem_u32(sb), aK = aQ + C::TENSOR_BYTES, aV = aQ + 2 * C::TENSOR_BYTES;
-    const long long u = u_begin + k;
-    const int h = (int)(u % p.heads);
-    const long long bs = u / p.heads;
-    const int s = (int)(bs % p.HW);
-    const int b = (int)(bs / p.HW);
 
     for (int mt = sub; mt < n_mt; mt += C::WPU) {
       // ---- S = Q K^T for rows mt*16 .. mt*16+15, all TP key columns
@@ -281,6 +289,10 @@ __global__ void __launch_bounds__(TimeCfg<D, TB>::LB_THREADS, 1)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
+    for (h += C::NP; h >= p.heads;) {
+      h -= p.heads;
+      if (++s == p.HW) { s = 0; ++b; }
+    }
   }
 }
 

@@ -159,8 +159,7 @@ enum : int { kSiteEmbA = 40, kSiteEmbW, kSiteEmbAcc, kSiteEmbDrain };
 __global__ void __launch_bounds__(kEmbThreads, 1)
     patch_embed_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmOut,
                        const EmbedParams p) {
-  const uintptr_t base = (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023);
-  unsigned char* sA = reinterpret_cast<unsigned char*>(base);            // 2 A buffers
+  unsigned char* sA = smem_base_1024();                                 // 2 A buffers
   unsigned char* sW = sA + 2 * kEmbATile;                                // weight ring
   unsigned char* sOut = sW + kEmbNW * kEmbWTile;                       // [epilogue warp][kEmbNStage] boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 4 * kEmbNStage * kEmbStage);

@@ -217,10 +217,17 @@ struct RopeShape {
   int ntens;          // 2: Q and K; 1: one tensor (K), passed in the Q slots
 };
 
-// Entry x of the per-axis (cos, sin) table: time [Tg][d_t/2], then height
-// [Hg][d_h/2] from off_h, then width [Wg][d_w/2] from off_w.  The angle is
-// pos * theta^(-2i/d) for pair i of a segment of width d, formed in float64;
-// cos and sin are rounded once to float32 (the snippet's complex64 cache).
+// (cos, sin) of pos * theta^(-2i/d) for pair i of a segment of width d: the
+// angle formed in float64, cos and sin rounded once to float32 (the snippet's
+// complex64 cache).
+__device__ __forceinline__ float2 rope_phasor(int pos, int i, int d, double theta) {
+  double sn, cn;
+  sincos((double)pos * (1.0 / pow(theta, (double)(2 * i) / (double)d)), &sn, &cn);
+  return make_float2((float)cn, (float)sn);
+}
+
+// Entry x of the position-major per-axis table: time [Tg][d_t/2], then height
+// [Hg][d_h/2] from off_h, then width [Wg][d_w/2] from off_w.
 __device__ __forceinline__ float2 rope_axis_entry(int x, int off_h, int off_w, int d_t, int d_h, int d_w,
                                                   double theta) {
   const int pt = d_t / 2, ph = d_h / 2, pw = d_w / 2;
@@ -228,19 +235,24 @@ __device__ __forceinline__ float2 rope_axis_entry(int x, int off_h, int off_w, i
   if (x < off_h) { pos = x / pt; i = x - pos * pt; d = d_t; }
   else if (x < off_w) { pos = (x - off_h) / ph; i = x - off_h - pos * ph; d = d_h; }
   else { pos = (x - off_w) / pw; i = x - off_w - pos * pw; d = d_w; }
-  double sn, cn;
-  sincos((double)pos * (1.0 / pow(theta, (double)(2 * i) / (double)d)), &sn, &cn);
-  return make_float2((float)cn, (float)sn);
+  return rope_phasor(pos, i, d, theta);
 }
 
-// The whole per-axis table in global memory, for kernels that look the pairs
-// up instead of building them (the attention kernel that rotates Q itself).
+// The whole per-axis table in global memory, pair-major (time [d_t/2][Tg],
+// then height [d_h/2][Hg], then width [d_w/2][Wg]), for kernels that look the
+// pairs of consecutive tokens up together (the attention kernel that rotates
+// Q itself): for one pair, neighbouring positions are neighbouring entries.
 __global__ void rope3d_table_kernel(float2* tab, int Tg, int Hg, int Wg, int d_t, int d_h, int d_w,
                                     double theta) {
   if (watchdog_tripped()) return;
   const int off_h = Tg * (d_t / 2), off_w = off_h + Hg * (d_h / 2), n = off_w + Wg * (d_w / 2);
-  for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < n; x += gridDim.x * blockDim.x)
-    tab[x] = rope_axis_entry(x, off_h, off_w, d_t, d_h, d_w, theta);
+  for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < n; x += gridDim.x * blockDim.x) {
+    int pos, i, d;
+    if (x < off_h) { i = x / Tg; pos = x - i * Tg; d = d_t; }
+    else if (x < off_w) { i = (x - off_h) / Hg; pos = x - off_h - i * Hg; d = d_h; }
+    else { i = (x - off_w) / Wg; pos = x - off_w - i * Wg; d = d_w; }
+    tab[x] = rope_phasor(pos, i, d, theta);
+  }
 }
 
 __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __nv_bfloat16* q_in, const __nv_bfloat16* k_in,

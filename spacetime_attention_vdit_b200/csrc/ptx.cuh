@@ -49,6 +49,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory window rounded up to a 1024-byte boundary (the
+// 128-byte swizzle pattern repeats every 1024 bytes).  Formed by pointer
+// arithmetic on the shared array itself, so that everything derived from it
+// stays in the shared address space for the compiler, which then emits
+// shared-memory loads and stores instead of generic ones.
+__device__ __forceinline__ unsigned char* smem_base_1024() {
+  return dyn_smem + ((1024u - (smem_u32(dyn_smem) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -153,6 +162,11 @@ __device__ __forceinline__ void regs_decrease() {
 // async-proxy reads (tensor-core operands, TMA stores).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier `id` over `count` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Named barrier `id` over `count` threads (whole warps) that also ANDs `pred`

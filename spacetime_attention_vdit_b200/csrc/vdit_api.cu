@@ -579,14 +579,16 @@ int vdit_attn_full_rope_q(const void* q, const void* k, const void* v, void* o, 
   if (norm_group != 0 && norm_group != head_dim) return VDIT_ERR_UNSUPPORTED;
   if (norm_group != 0 && (!(eps >= 0.f) || !std::isfinite(eps))) return VDIT_ERR_SHAPE;
   if (!aligned16(rope_table) || (wq && !aligned16(wq))) return VDIT_ERR_ALIGN;
-  if (rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w) > 0x7fffffffLL) return VDIT_ERR_SHAPE;
+  // the kernel stages the table in one K/V ring stage: 128 x head_dim bf16
+  if (rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w) * 8 > 128LL * head_dim * 2) return VDIT_ERR_UNSUPPORTED;
   AttnParams r{};
   r.rope_tab = reinterpret_cast<const float2*>(rope_table);
   r.wq = wq;
-  r.rope_hg = Hg; r.rope_wg = Wg;
-  r.rope_pt = d_t / 2; r.rope_ph = d_h / 2; r.rope_pw = d_w / 2;
+  r.rope_tg = Tg; r.rope_hg = Hg; r.rope_wg = Wg;
+  r.rope_pt = d_t / 2; r.rope_ph = d_h / 2;
   r.rope_off_h = Tg * (d_t / 2);
   r.rope_off_w = r.rope_off_h + Hg * (d_h / 2);
+  r.rope_n = (int)rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w);
   r.norm = norm_group != 0;
   r.eps = eps;
   r.inv_d = 1.f / (float)head_dim;
