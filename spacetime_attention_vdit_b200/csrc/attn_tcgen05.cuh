@@ -46,6 +46,8 @@
 
 #include <math.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace vdit {
@@ -215,6 +217,10 @@ __device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* 
   const bool live = active && i < p.L;          // rows past the sequence stay zero
   // every softmax thread takes part, whatever its tile: the barrier counts 256
   for (int x = (int)threadIdx.x; x < p.rope_n; x += 256) tabs[x] = __ldg(p.rope_tab + x);
+  // the norm's weights (1 without a weight vector) follow the table
+  float* wv = reinterpret_cast<float*>(tabs + p.rope_n);
+  if (p.norm)
+    for (int x = (int)threadIdx.x; x < D; x += 256) wv[x] = p.wq != nullptr ? __ldg(p.wq + x) : 1.f;
   named_bar_sync(3, 256);
   int bt = 0, bh = 0, bw = 0;
   if (live) {
@@ -261,30 +267,53 @@ __device__ __forceinline__ bool rope_q_rows(const AttnParams& p, unsigned char* 
         for (int k = 0; k < o; ++k) a[k] = a[k] + a[k + o];
       nscale = rsqrtf(fmaf(a[0], p.inv_d, p.eps));
     }
+    // Half a row at a time: every load of the half (its Q chunks and their
+    // pairs' (cos, sin)) is issued before its first store, which the compiler
+    // may not move a later shared-memory load above: one load latency per half
+    // instead of one per chunk.  The loop is instantiated with and without the
+    // norm so that no branch splits it.
+    auto rotate = [&](auto with_norm) {
+      constexpr bool kNorm = decltype(with_norm)::value;
+      constexpr int HALF = NCH / 2;
 #pragma unroll
-    for (int cc = 0; cc < NCH; ++cc) {
-      uint4* dst = chunk(cc);
-      const uint4 x = *dst;
-      uint32_t u[4] = {x.x, x.y, x.z, x.w};
+      for (int c0 = 0; c0 < NCH; c0 += HALF) {
+        uint4 xv[HALF];
+        float2 cv[HALF][4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&u[m]);
-        float x0 = __low2float(pr), x1 = __high2float(pr);
-        if (p.norm) {
-          const float w0 = p.wq != nullptr ? __ldg(p.wq + cc * 8 + 2 * m) : 1.f;
-          const float w1 = p.wq != nullptr ? __ldg(p.wq + cc * 8 + 2 * m + 1) : 1.f;
-          x0 = __fmul_rn(__fmul_rn(x0, nscale), w0);
-          x1 = __fmul_rn(__fmul_rn(x1, nscale), w1);
+        for (int u = 0; u < HALF; ++u) xv[u] = *chunk(c0 + u);
+#pragma unroll
+        for (int u = 0; u < HALF; ++u)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int pi = (c0 + u) * 4 + m;
+            cv[u][m] = tabs[pi < p.rope_pt ? bt + pi * p.rope_tg
+                                           : (pi < p.rope_pt + p.rope_ph ? bh + pi * p.rope_hg : bw + pi * p.rope_wg)];
+          }
+#pragma unroll
+        for (int u = 0; u < HALF; ++u) {
+          const int cc = c0 + u;
+          uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w[m]);
+            float x0 = __low2float(pr), x1 = __high2float(pr);
+            if constexpr (kNorm) {
+              x0 = __fmul_rn(__fmul_rn(x0, nscale), wv[cc * 8 + 2 * m]);
+              x1 = __fmul_rn(__fmul_rn(x1, nscale), wv[cc * 8 + 2 * m + 1]);
+            }
+            const float2 c = cv[u][m];
+            const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
+            const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
+            w[m] = pack_bf16x2(re, im);
+          }
+          *chunk(cc) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        const int pi = cc * 4 + m;
-        const float2 c = tabs[pi < p.rope_pt ? bt + pi * p.rope_tg
-                                             : (pi < p.rope_pt + p.rope_ph ? bh + pi * p.rope_hg : bw + pi * p.rope_wg)];
-        const float re = __fsub_rn(__fmul_rn(x0, c.x), __fmul_rn(x1, c.y));
-        const float im = __fadd_rn(__fmul_rn(x0, c.y), __fmul_rn(x1, c.x));
-        u[m] = pack_bf16x2(re, im);
       }
-      *dst = make_uint4(u[0], u[1], u[2], u[3]);
-    }
+    };
+    if (p.norm)
+      rotate(std::true_type{});
+    else
+      rotate(std::false_type{});
   }
   // the rewritten rows, and this thread's share of the table copy, are ordered
   // before the tensor core's reads and the TMA's next writes there; then the

@@ -579,8 +579,10 @@ int vdit_attn_full_rope_q(const void* q, const void* k, const void* v, void* o, 
   if (norm_group != 0 && norm_group != head_dim) return VDIT_ERR_UNSUPPORTED;
   if (norm_group != 0 && (!(eps >= 0.f) || !std::isfinite(eps))) return VDIT_ERR_SHAPE;
   if (!aligned16(rope_table) || (wq && !aligned16(wq))) return VDIT_ERR_ALIGN;
-  // the kernel stages the table in one K/V ring stage: 128 x head_dim bf16
-  if (rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w) * 8 > 128LL * head_dim * 2) return VDIT_ERR_UNSUPPORTED;
+  // the kernel stages the table, then the norm's head_dim weights, in one K/V
+  // ring stage: 128 x head_dim bf16
+  if (rope_table_entries(Tg, Hg, Wg, d_t, d_h, d_w) * 8 + head_dim * 4 > 128LL * head_dim * 2)
+    return VDIT_ERR_UNSUPPORTED;
   AttnParams r{};
   r.rope_tab = reinterpret_cast<const float2*>(rope_table);
   r.wq = wq;
