@@ -65,7 +65,7 @@ struct AttnCfg {
   static constexpr int TILE_BYTES = BM * D * 2;
   static constexpr int NK = D >= 128 ? 3 : 4;                  // K ring stages
   static constexpr int NV = D >= 128 ? 2 : (D >= 64 ? 3 : 4);  // V ring stages
-  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 3 * NQ + 1;
+  static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 4 * NQ + 1;
   static constexpr int SMEM_BYTES = 1024 + (NQ + NK + NV) * TILE_BYTES + NBARS * 8 + 16;
   static constexpr int THREADS = 384;                          // three warpgroups
   static constexpr int TMA_WARP = 8, MMA_WARP = 9;
@@ -345,7 +345,8 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
   uint64_t* p_full = s_full + C::NQ;       // [NQ]
   uint64_t* drain = p_full + C::NQ;        // every UMMA of the CTA has finished
   uint64_t* q_ready = drain + 1;           // [NQ] Q tile rotated in place (kRopeQ)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + C::NQ);
+  uint64_t* o_done = q_ready + C::NQ;      // [NQ] the tile's last P.V (and all before it) finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + C::NQ);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -370,6 +371,7 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);           // one elected lane per softmax warp
       mbar_init(&q_ready[i], 4);
+      mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -504,6 +506,10 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
           if (!ok) break;
           tc_fence_after();
           pv(i, j);
+          // with few key tiles the epilogue weighs: each tile's starts as soon
+          // as its own last P.V is done (long sequences keep the one drain,
+          // which measured faster there)
+          if (kStageO && j + 1 == n) umma_commit(&o_done[i]);
           if (j + 1 < n) {
             if (i == 0) ok = mbar_wait(&k_full[(j + 1) % C::NK], ((j + 1) / C::NK) & 1, kSiteKFull);
             if (!ok) break;
@@ -637,13 +643,14 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
         }
       }
     } else {
-      // O / l is staged in this tile's Q buffer (every UMMA, the QK^T ones that
-      // read Q included, has finished once `drain` fires) in the layout of the
+      // O / l is staged in this tile's Q buffer (every UMMA that reads it has
+      // finished once o_done fires: UMMAs complete in issue order, and the
+      // tile's last Q.K^T precedes its last P.V) in the layout of the
       // Q tensor map; then one thread sends the tile with one TMA store per
       // D-block, rows past the sequence end clipped, so whole 128-byte lines
       // leave the SM instead of a 16-byte piece per row and lane
       bool good = ok;
-      if (good) good = warp_wait(drain, 0, kSiteODone);
+      if (good) good = warp_wait(&o_done[tile], 0, kSiteODone);
       if (good) {
         tc_fence_after();
         const int i = q0 + tile * C::BM + row;      // position in the sequence
