@@ -326,11 +326,11 @@ def attn_full_rope_q(q, k, v, grid, table, split=None, wq=None, norm_group: int 
     ``table`` (:func:`rope_3d_table` of the same grid and split).  K must already
     be normalised and rotated (:func:`rope_3d` / :func:`qk_norm_rope_3d` with
     ``q=None``).  ``lse=True`` also returns [B, heads, L]."""
+    Tg, Hg, Wg = grid
+    if q.dim() != 4 or Tg * Hg * Wg != q.shape[1]:
+        raise ValueError("grid does not match the sequence length")
     out, lse_t, lse_p = _attn_io(q, k, v, out, lse)
     B, L, Hh, D = q.shape
-    Tg, Hg, Wg = grid
-    if Tg * Hg * Wg != L:
-        raise ValueError("grid does not match the sequence length")
     d_t, d_h, d_w = default_split(D) if split is None else split
     wp = None
     if wq is not None:

@@ -214,6 +214,13 @@ def test_binding_refuses_cpu_tensors(L):
         v.attn_full(q, q, q)
     with pytest.raises(ValueError, match="CUDA"):
         v.patchify_3d(torch.zeros((1, 1, 1, 2, 2)))
+    with pytest.raises(ValueError, match="CUDA"):
+        v.rope_3d(None, q, (1, 2, 4), (12, 10, 10))
+    tab = torch.zeros((1 * 6 + 2 * 5 + 4 * 5, 2), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        v.attn_full_rope_q(q, q, q, (1, 2, 4), tab, (12, 10, 10))
+    with pytest.raises(ValueError, match="grid"):
+        v.attn_full_rope_q(q, q, q, (1, 2, 5), tab, (12, 10, 10))
 
 
 def test_build_command_targets_sm100a():
