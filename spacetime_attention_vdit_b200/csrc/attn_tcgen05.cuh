@@ -126,13 +126,15 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// 2^x on the FMA pipe, for x <= 8: x = n + f with n = rint(x) (the 1.5 * 2^23
-// rounding constant) and |f| <= 1/2; 2^f from a cubic fitted here by
-// relative-error least squares on [-1/2, 1/2] (max relative error 7.8e-5, below
-// half a bf16 ulp); n is added to the exponent field.  Below -125 the result is
+// 2^x on the FMA pipe: x = n + f with n = rint(x) (the 1.5 * 2^23 rounding
+// constant) and |f| <= 1/2; 2^f from a cubic fitted here by relative-error
+// least squares on [-1/2, 1/2] (max relative error 7.8e-5, below half a bf16
+// ulp); n is added to the exponent field.  x is clamped to at most 8 (so x > 8
+// gives 2^8 within the fit's error, which the softmax's sum test relies on: it
+// is far above the test's 2^7); below -125 the result is
 // 0, like the MUFU's flushed 2^x there, and a masked score (-inf) gives exactly 0.
 __device__ __forceinline__ float2 ex2_fma2(float2 x) {
-  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  const float2 xc = make_float2(fminf(fmaxf(x.x, -125.f), 8.f), fminf(fmaxf(x.y, -125.f), 8.f));
   const float2 rnd = make_float2(12582912.f, 12582912.f);
   const float2 t = fadd2(xc, rnd);                                         // rnd + rint(x)
   const float2 f = fadd2(xc, ffma2(t, make_float2(-1.f, -1.f), rnd));     // x - rint(x)
@@ -560,30 +562,51 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e >= valid) s[c][e] = __float_as_uint(-INFINITY);
       }
-      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four max chains
+      // the tile's row max, in log2 units
+      auto tile_max = [&]() -> float {
+        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four max chains
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          mp[(e >> 1) & 3] = fmax3(mp[(e >> 1) & 3], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-      const float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]), mp[3]);
-      const float m_new = mx * p.scale_log2;
+          for (int e = 0; e < 32; e += 2)
+            mp[(e >> 1) & 3] = fmax3(mp[(e >> 1) & 3], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+        return fmaxf(fmax3(mp[0], mp[1], mp[2]), mp[3]) * p.scale_log2;
+      };
+      // P = 2^(s - m_use) over this tile's own score columns; returns the row's sum
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      auto exps = [&]() -> float {
+        float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};   // four independent packed sum chains
+        exp_tile(s, t_s, sc2, make_float2(-m_use, -m_use), sp);
+        const float2 s01 = fadd2(fadd2(sp[0], sp[1]), fadd2(sp[2], sp[3]));
+        return s01.x + s01.y;
+      };
+      // The max in use only moves when a tile raises it by more than 8 (log2
+      // units; exact: every P stays <= 2^8 and O / l is unchanged).  After the
+      // first tile the exponentials are taken against the max in use straight
+      // away, and the tile's max is computed only when the tile's sum of P
+      // reaches 2^7, which a P above 2^7 implies (the FMA-pipe exponential
+      // saturates just below 2^8 for larger arguments, well above 2^7); then,
+      // if the max must move, P is taken again.  Once a row's first tiles are
+      // in, its scores rarely climb that far, so the max pass leaves the
+      // softmax chain.
       float alpha = 1.f;
       bool rescale = false;
-      if (j == 0) {
-        m_use = m_new;
-      } else if (m_new > m_use + 8.f) {
-        alpha = ex2_approx(m_use - m_new);
-        m_use = m_new;
-        rescale = true;
+      if (j == 0) m_use = tile_max();
+      float lt = exps();
+      if (j > 0 && __any_sync(0xffffffffu, !(lt < 128.f))) {
+        const float m_new = tile_max();
+        rescale = m_new > m_use + 8.f;
+        if (__any_sync(0xffffffffu, rescale)) {   // the stores of P are warp-wide: the warp redoes them
+          if (rescale) {
+            alpha = ex2_approx(m_use - m_new);
+            m_use = m_new;
+          }
+          tmem_st_wait();       // the first stores of P have landed before they are overwritten
+          lt = exps();
+        }
       }
-      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-      const float2 nm2 = make_float2(-m_use, -m_use);
-      float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f)};   // four independent packed sum chains
-      exp_tile(s, t_s, sc2, nm2, sp);     // P over this tile's own score columns
-      const float2 s01 = fadd2(fadd2(sp[0], sp[1]), fadd2(sp[2], sp[3]));
-      l_sum = l_sum * alpha + (s01.x + s01.y);
+      l_sum = l_sum * alpha + lt;
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

@@ -1,9 +1,11 @@
 """Host check of the FMA-pipe 2^x used for a share of the softmax exponentials
 (ex2_fma2 in the attention kernel): the cubic's coefficients, read from the
 source, and the float32 steps of the function emulated here, stay within the
-stated relative error of 2^x over the whole range the softmax feeds it
-(x = s * scale * log2 e - m <= 8, m the running row maximum), and give 0 below
--125 and for a masked score (-inf)."""
+stated relative error of 2^x over the range where the softmax keeps its
+results (x = s * scale * log2 e - m <= 8, m the max in use), give 2^8 (within
+the fit's error) above it, far above the 2^7 at which the softmax's sum test
+recomputes the max,
+and give 0 below -125 and for a masked score (-inf)."""
 import os
 import re
 
@@ -29,7 +31,7 @@ def ex2_fma_emulated(x):
     """The kernel's steps in float32 (fma rounded once, as the hardware does)."""
     c3, c2, c1, c0 = coefficients()
     x = np.asarray(x, dtype=np.float32)
-    xc = np.maximum(x, np.float32(-125.0))
+    xc = np.minimum(np.maximum(x, np.float32(-125.0)), np.float32(8.0))
     rnd = np.float32(12582912.0)
     t = (xc + rnd).astype(np.float32)
     f = (xc.astype(np.float64) + (rnd.astype(np.float64) - t.astype(np.float64))).astype(np.float32)
@@ -64,3 +66,14 @@ def test_emulated_function_matches_exp2_over_the_softmax_range():
 def test_below_range_and_masked_scores_give_zero():
     x = np.array([-125.001, -126.0, -300.0, -1e30, -np.inf], dtype=np.float32)
     assert np.all(ex2_fma_emulated(x) == 0.0)
+
+
+def test_above_eight_saturates_at_two_to_the_eight():
+    """A score above the max in use by more than 8 (log2 units) comes out as 2^8
+    (within the fit's error), so the tile's sum of P reaches the softmax's 2^7
+    test and the max is recomputed: such a value is never kept."""
+    x = np.array([8.0, 8.0001, 9.0, 20.0, 127.0, 1e30, np.inf], dtype=np.float32)
+    got = ex2_fma_emulated(x).astype(np.float64)
+    assert np.abs(got[0] / 256.0 - 1.0) < 1.2e-4
+    assert np.all(got[1:] == got[0]) and got[0] > 2.0 * 128.0 * (1.0 - 1e-3)
+
