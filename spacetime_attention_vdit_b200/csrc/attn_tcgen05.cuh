@@ -544,7 +544,8 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
     if constexpr (kRopeQ)
       ok = rope_q_rows<D>(p, sQ + tile * C::TILE_BYTES, reinterpret_cast<float2*>(sV + C::TILE_BYTES), q_full,
                           &q_ready[tile], ok, q0 + tile * C::BM + row, row, bb, lane);
-    for (int j = 0; j < n && ok; ++j) {
+    int kt = j0;                                  // key tile of this iteration: (j + j0) mod n, stepped
+    for (int j = 0; j < n && ok; ++j, kt = (kt + 1 == n) ? 0 : kt + 1) {
       if (!warp_wait(&s_full[tile], j & 1, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[4][32];
@@ -554,7 +555,7 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_fence(s[c]);
 
-      const int valid = p.Lk - ((j + j0) % n) * C::BN;  // keys of this tile inside the sequence
+      const int valid = p.Lk - kt * C::BN;          // keys of this tile inside the sequence
       if (valid < C::BN) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -591,12 +592,11 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
       // in, its scores rarely climb that far, so the max pass leaves the
       // softmax chain.
       float alpha = 1.f;
-      bool rescale = false;
       if (j == 0) m_use = tile_max();
       float lt = exps();
       if (j > 0 && __any_sync(0xffffffffu, !(lt < 128.f))) {
         const float m_new = tile_max();
-        rescale = m_new > m_use + 8.f;
+        const bool rescale = m_new > m_use + 8.f;
         if (__any_sync(0xffffffffu, rescale)) {   // the stores of P are warp-wide: the warp redoes them
           if (rescale) {
             alpha = ex2_approx(m_use - m_new);
@@ -604,21 +604,20 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
           }
           tmem_st_wait();       // the first stores of P have landed before they are overwritten
           lt = exps();
+          // O follows the max in use (alpha is 1 for the rows whose max stayed)
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_ld_wait();
+            tmem_ld_fence(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
         }
       }
       l_sum = l_sum * alpha + lt;
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + c * 32, o);
-          tmem_ld_wait();
-          tmem_ld_fence(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(t_o + c * 32, o);
-        }
-      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
