@@ -29,10 +29,12 @@
 // [128 i, 128 i + 128), O of tile i at [256 + 128 i, ...).
 //
 // Softmax per tile and row: running max m kept unless a new tile raises it by
-// more than 2^8 (exact rescaling rule: P stays below 2^8 and O/l is unchanged);
-// P = 2^(s * scale * log2e - m) rounded to bf16, one pair in kFmaPairEvery
-// exponentiated on the FMA pipe to unload the MUFU; O rescaled in TMEM only
-// when m moved; at the end O / l and the row's log-sum-exp are written out.
+// more than 8 in log2 units (exact rescaling rule: P stays at most 2^8 and O/l
+// is unchanged), the tile's max computed only on the first tile and when the
+// tile's sum of P reaches 2^7; P = 2^(s * scale * log2e - m) rounded to bf16,
+// one pair in kFmaPairEvery exponentiated on the FMA pipe to unload the MUFU;
+// O rescaled in TMEM only when m moved; at the end O / l and the row's
+// log-sum-exp are written out.
 // kStageO picks how O leaves the SM: false, each thread stores its own row
 // with 16-byte stores; true, the rows are staged in the tile's Q buffer and
 // sent with TMA stores, which pays off when a CTA sweeps only a few key tiles
