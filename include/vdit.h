@@ -276,8 +276,11 @@ int vdit_attn_full(const void* q, const void* k, const void* v, void* o, float* 
  * (weight 1) or device float32 [head_dim], 16-byte aligned.
  * Errors: VDIT_ERR_NULL, VDIT_ERR_SHAPE (also: the split as for vdit_rope_3d,
  * eps negative or not finite when normalising), VDIT_ERR_ALIGN,
- * VDIT_ERR_UNSUPPORTED (head_dim; norm_group other than 0 or head_dim),
- * VDIT_ERR_CUDA.
+ * VDIT_ERR_UNSUPPORTED (head_dim; norm_group other than 0 or head_dim; a
+ * table of n pairs with 8*n + 4*head_dim above 256*head_dim bytes, the
+ * shared-memory stage the kernel stages the table and the weights in: 4,032
+ * pairs at head_dim 128, more than Tg*22 + (Hg + Wg)*21 for every grid the
+ * sources use), VDIT_ERR_CUDA.
  * Watchdog: device-wide (see the conventions above).
  */
 int vdit_attn_full_rope_q(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -126,6 +126,11 @@ def test_attn_full_rope_q_validation(L):
     assert attn_rope(L, tab=MIS) == ALIGN
     assert attn_rope(L, group=128, wq=MIS) == ALIGN
     assert attn_rope(L, k=MIS) == ALIGN
+    # the table and the weights are staged in one K/V stage: 8 n + 4 D <= 256 D
+    # bytes, 4,032 pairs at D = 128 (a call that passed every check would
+    # launch, so only the refused side is called here)
+    assert L.vdit_rope_3d_table_entries(182, 1, 1, 128, 44, 42, 42) == 4046
+    assert attn_rope(L, grid=(182, 1, 1), split=(44, 42, 42), B=1) == UNSUP
 
 
 def norm_rope(L, q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, wq=None, wk=None, group=128, eps=1e-6, B=1, Tg=2, Hg=3,
