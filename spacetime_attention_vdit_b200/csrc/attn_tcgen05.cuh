@@ -379,6 +379,19 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
     }
     mbar_init(drain, 1);
     fence_mbar_init();
+    // Q and the first K tile, which the first Q.K^T waits for, are requested
+    // here, before the CTA-wide set-up (TMEM allocation, the barrier), which
+    // their latency then covers; the producer continues from K_1
+    mbar_arrive_expect_tx(q_full, nq * C::TILE_BYTES);
+    for (int i = 0; i < nq; ++i)
+#pragma unroll
+      for (int db = 0; db < C::NDB; ++db)
+        tma_load_5d(sQ + i * C::TILE_BYTES + db * C::DB_BYTES, &tmQ, q_full, db * C::DBLK, h, c_site,
+                    q0 + i * C::BM, c_batch);
+    mbar_arrive_expect_tx(&k_full[0], C::TILE_BYTES);
+#pragma unroll
+    for (int db = 0; db < C::NDB; ++db)
+      tma_load_5d(sK + db * C::DB_BYTES, &tmK, &k_full[0], db * C::DBLK, h, c_site, j0 * C::BN, c_batch);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -396,16 +409,8 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
   if (warp == C::TMA_WARP) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, nq * C::TILE_BYTES);
-      for (int i = 0; i < nq; ++i)
-#pragma unroll
-        for (int db = 0; db < C::NDB; ++db)
-          tma_load_5d(sQ + i * C::TILE_BYTES + db * C::DB_BYTES, &tmQ, q_full, db * C::DBLK, h, c_site,
-                      q0 + i * C::BM, c_batch);
-      int k_issued = 0, v_issued = 0;
+      int k_issued = 1, v_issued = 0;     // Q and K_0 were requested during set-up
       auto load_k = [&](int j) -> bool {
         const int st = j % C::NK;
         if (j >= C::NK && !mbar_wait(&k_empty[st], ((j / C::NK) - 1) & 1, kSiteKEmpty)) return false;
@@ -429,7 +434,7 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tmQ, const CUte
         return true;
       };
       // K runs one tile ahead of V: K_0, K_1, V_0, K_2, V_1, ...
-      bool ok = load_k(0);
+      bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n) ok = load_k(j + 1);
         if constexpr (kRopeQ) {
