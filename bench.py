@@ -52,6 +52,8 @@ sys.path.insert(0, ROOT)
 METRIC = "attention TFLOP/s and ms/layer at 32,760 tokens; % of B200 dense BF16 peak"
 
 TEXT_TOKENS = 512          # prompt tokens the video tokens cross-attend to (towardsai section 5)
+E2E_SETS = 3               # device buffer sets the end-to-end pipeline rotates through
+E2E_MIN_STEPS = 64         # end-to-end steps timed at least (fill and drain included)
 
 WORKLOADS = {
     # name: (B, T latent frames, H latent, W latent, heads, head_dim, description)
@@ -604,17 +606,20 @@ def main():
     # ---- end to end through the public API with host buffers
     # Every step copies its inputs in from pinned host memory and its results
     # back out.  The copies of one step overlap the compute of its neighbours:
-    # three streams (host->device, compute, device->host) and two device buffer
-    # sets, as a serving loop would run them; the timed region spans the first
-    # input copy to the last output copy, pipeline fill and drain included.
+    # three streams (host->device, compute, device->host) and three device
+    # buffer sets, as a serving loop would run them (a step's input copy may
+    # start once the step three back has been computed, so a late copy does not
+    # stall the compute stream); the timed region spans the first input copy to
+    # the last output copy, pipeline fill and drain included.
     e2e = None
     if not args.no_e2e:
         sets = [dict(lat=lat, q=q, k=k, v=v, tok=tok, qr=qr, kr=kr, o_full=o_full, o_time=o_time,
                      o_space=o_space)]
-        sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
+        for _ in range(E2E_SETS - 1):
+            sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
         out_names = ("tok", "o_full", "o_time", "o_space")
         outs_h = [[torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype).pin_memory() for n in out_names]
-                  for _ in range(2)]
+                  for _ in range(E2E_SETS)]
         h2d = sum(t.numel() * t.element_size() for t in (lat_h, q_h, k_h, v_h))
         d2h = sum(sets[0][n].numel() * sets[0][n].element_size() for n in out_names)
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -630,20 +635,20 @@ def main():
         def run_pipeline(n_steps, first=None, last=None):
             ev_in, ev_comp, ev_out = {}, {}, {}
             for t in range(n_steps):
-                bs, oh = sets[t % 2], outs_h[t % 2]
+                bs, oh = sets[t % E2E_SETS], outs_h[t % E2E_SETS]
                 with torch.cuda.stream(s_in):
                     if t == 0 and first is not None:
                         first.record(s_in)
-                    if t >= 2:
-                        s_in.wait_event(ev_comp[t - 2])         # the set's inputs are consumed
+                    if t >= E2E_SETS:
+                        s_in.wait_event(ev_comp[t - E2E_SETS])  # the set's inputs are consumed
                     for name, hsrc in (("lat", lat_h), ("q", q_h), ("k", k_h), ("v", v_h)):
                         bs[name].copy_(hsrc, non_blocking=True)
                     ev_in[t] = torch.cuda.Event()
                     ev_in[t].record(s_in)
                 with torch.cuda.stream(s_comp):
                     s_comp.wait_event(ev_in[t])
-                    if t >= 2:
-                        s_comp.wait_event(ev_out[t - 2])        # the set's outputs are read out
+                    if t >= E2E_SETS:
+                        s_comp.wait_event(ev_out[t - E2E_SETS])  # the set's outputs are read out
                     set_step(bs)
                     ev_comp[t] = torch.cuda.Event()
                     ev_comp[t].record(s_comp)
@@ -656,8 +661,10 @@ def main():
             if last is not None:
                 last.record(s_out)
 
-        run_pipeline(2)
-        e_steps = max(4, min(args.steps, 16))
+        run_pipeline(E2E_SETS)
+        # a serving loop runs without end: enough steps that the fill and drain
+        # (one step's input copy and one step's output copy) weigh little
+        e_steps = min(max(args.steps, E2E_MIN_STEPS), 4 * E2E_MIN_STEPS)
         barrier()
         torch.cuda.synchronize(dev)
         s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -668,11 +675,30 @@ def main():
         rc, flags = vd.device_status()
         if rc != 0:
             raise RuntimeError(f"kernel watchdog tripped in the end-to-end leg: flags {flags:#x}")
+        # each direction's copies alone, on an idle device: the rate the
+        # pipeline cannot beat when the copies take longer than the kernels
+        copy_ms = {}
+        for direction in ("h2d", "d2h"):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s_in):
+                a.record(s_in)
+                if direction == "h2d":
+                    for name, hsrc in (("lat", lat_h), ("q", q_h), ("k", k_h), ("v", v_h)):
+                        sets[1][name].copy_(hsrc, non_blocking=True)
+                else:
+                    for hbuf, name in zip(outs_h[1], out_names):
+                        hbuf.copy_(sets[1][name], non_blocking=True)
+                b.record(s_in)
+            torch.cuda.synchronize(dev)
+            copy_ms[direction] = max_over_ranks(a.elapsed_time(b))
         e2e = {"value": job_throughput(world, flops_step, e_steps, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms / e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": e_steps,
-               "pipelined": "host->device, compute and device->host on three streams, two device buffer sets"}
-        del sets[1]
+               "h2d_ms_alone": copy_ms["h2d"], "d2h_ms_alone": copy_ms["d2h"],
+               "h2d_gb_s": h2d / (copy_ms["h2d"] * 1e-3) / 1e9, "d2h_gb_s": d2h / (copy_ms["d2h"] * 1e-3) / 1e9,
+               "pipelined": (f"host->device, compute and device->host on three streams, {E2E_SETS} device "
+                             "buffer sets; fill and drain inside the timed region")}
+        del sets[1:]
 
     # ---- roofline of the dominant kernel (full attention)
     peaks, peaks_kind = measured_peaks()
