@@ -217,6 +217,24 @@ def oracle_sample(d, budget_s, seed=0):
                       f"space pass over {HW} keys and time pass over {T} keys, float64 NumPy", done_rows
 
 
+def oracle_full_small(seed=0):
+    """Time the float64 oracle's full attention over every query row of the
+    17-frame 480p clip (7,800 tokens x 12 heads x 128): small enough to run whole."""
+    import synthetic
+    from oracle import reference as ref
+
+    B, T, H, W, heads, D, _ = WORKLOADS["480p17"]
+    L = T * (H // PATCH[1]) * (W // PATCH[2])
+    q, k, v = synthetic.qkv_bf16(B, L, heads, D, seed=seed)
+    qf, kf, vf = (synthetic.bf16_bits_to_f64(x) for x in (q, k, v))
+    t0 = time.perf_counter()
+    ref.attention(qf, kf, vf)
+    el = time.perf_counter() - t0
+    flops = 4 * B * heads * L * L * D
+    return {"workload": "480p17", "what": f"full attention, every one of {L} rows x {heads} heads, float64 NumPy",
+            "s": el, "tflops": flops / el / 1e12}
+
+
 def oracle_rates(d, flops, seconds, rows):
     """Measured oracle rows per second, and the time a whole step would take at the
     measured FLOP rate (extrapolated: the oracle never runs a whole step)."""
@@ -844,7 +862,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, s, desc, r = oracle_sample(d, 15.0)
         cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": desc + f"; {s:.1f} s", **oracle_rates(d, f, s, r)}
+               "sample": desc + f"; {s:.1f} s", **oracle_rates(d, f, s, r),
+               "whole_small_clip": oracle_full_small()}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
